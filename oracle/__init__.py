@@ -1,0 +1,13 @@
+"""Float64 CPU oracle (test infrastructure only; see ``sts_oracle``)."""
+
+from .sts_oracle import (  # noqa: F401
+    RowFilter,
+    backward,
+    filter_row,
+    filter_rows,
+    forward,
+    logit_grad,
+    row_gaps,
+    sample_rows,
+    scaled_logits,
+)
