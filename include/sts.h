@@ -1,0 +1,174 @@
+/*
+ * sts.h -- C ABI of the B200 (sm_100a) sampling-transform scoring core.
+ *
+ * The operation (defined in "Consolidate sampling-transform scoring on one
+ * shared chunked core; implement top-k/top-p/min-p replay for generic
+ * ce_modes", xorl pull request 74, section "What this PR does", items 1, 2
+ * and 4):
+ *
+ *   for every row t (a scored token) with hidden state H[t,:]:
+ *     z_i   = sum_j H[t,j] * W[i,j]            bf16 operands, fp32 accumulate
+ *     s_i   = z_i / tau_t                      per-row temperature, applied
+ *                                              after the projection, IEEE fp32
+ *                                              division
+ *     S_t   = top-k  (k_t)  then top-p (p_t, measured on the top-k-renormalised
+ *             mass, inclusive crossing)  then min-p (mu_t, against the
+ *             unfiltered row max); ties ordered by token id
+ *     logprob_t = min(s_y - log sum_{i in S_t} exp(s_i), 0)   if y_t in S_t
+ *               = -inf                                         otherwise
+ *
+ *   and the closed-form backward (recompute, only per-row scalars kept):
+ *     dz_i = g_t * (1[i == y_t] - exp(s_i - LSE_S) * 1[i in S_t]) / tau_t
+ *            (a zero row when y_t is outside S_t)
+ *     dH = dZ . W,   dW = dZ^T . H
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *     owned by the caller. The library allocates no device memory: scratch
+ *     comes from the caller's workspace (size from sts_workspace_bytes).
+ *   - Calls are asynchronous on the given stream. Errors a host can see
+ *     (NULL pointers, bad shapes, small workspace, wrong device) return
+ *     immediately and launch nothing. Errors that depend on row values
+ *     (temperature, top_p, min_p, target) are written to a status word in
+ *     the workspace; sts_get_status() reads it.
+ *   - Rows whose values are invalid produce logprob = NaN and a zero
+ *     gradient; other rows are unaffected.
+ *   - A target outside its row's support is not an error: logprob = -inf
+ *     and the row's gradient is zero (item 4 of the page).
+ *   - Only bf16 H and W are accepted (an fp8 head is rejected one level up,
+ *     in the Python binding, with STS_ERR_DTYPE).
+ *   - Layouts: H [T, d] and W [V, d] row-major bf16 (nn.Linear weight
+ *     layout); dH [T, d] and dW [V, d] row-major fp32; per-row arrays [T].
+ *   - Alignment: d must be a multiple of 8 (16-byte TMA strides); H, W, dH,
+ *     dW and the scaled-logits buffer must be 16-byte aligned; the workspace
+ *     must be 256-byte aligned (STS_ERR_WORKSPACE otherwise).
+ *   - Device: compute capability 10.0 (B200, sm_100a) only.
+ */
+#ifndef STS_H_
+#define STS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define STS_ABI_VERSION 1
+
+/* cudaStream_t without pulling in the CUDA headers (same opaque type). */
+typedef struct CUstream_st* sts_stream_t;
+
+typedef enum {
+  STS_OK = 0,
+  STS_ERR_NULL = 1,             /* a required pointer is NULL */
+  STS_ERR_SHAPE = 2,            /* T, d, V, chunk sizes, alignment, or a
+                                   metadata length != T (validated, never
+                                   truncated: "Self-review pass") */
+  STS_ERR_DTYPE = 3,            /* operand dtype other than bf16 (binding) */
+  STS_ERR_TEMPERATURE = 4,      /* some row has tau not finite or <= 0 */
+  STS_ERR_TOP_K = 5,            /* reserved: every int32 top_k is valid */
+  STS_ERR_TOP_P = 6,            /* some row has top_p not in (0, 1] */
+  STS_ERR_MIN_P = 7,            /* some row has min_p not in [0, 1] */
+  STS_ERR_TARGET = 8,           /* some row has target not in [0, V) */
+  STS_ERR_WORKSPACE = 9,        /* workspace NULL, too small or misaligned */
+  STS_ERR_OVERFLOW = 10,        /* an internal bound was exceeded */
+  STS_ERR_TIMEOUT = 11,         /* a bounded device wait gave up */
+  STS_ERR_CUDA = 12,            /* a CUDA runtime/driver call failed */
+  STS_ERR_UNSUPPORTED_ARCH = 13 /* current device is not sm_100 */
+} sts_status;
+
+/* Problem shape. */
+typedef struct {
+  int64_t T;           /* rows (scored tokens), >= 1 */
+  int64_t d;           /* hidden size, >= 8, multiple of 8 */
+  int64_t V;           /* vocabulary size, >= 1, < 2^31 */
+  int64_t vocab_chunk; /* backward vocab chunk (multiple of 256); 0: default */
+  int64_t row_chunk;   /* forward row chunk (multiple of 128); 0: default */
+} sts_shape;
+
+/* Per-row transform metadata ("What this PR does", items 1-3). */
+typedef struct {
+  int64_t len;              /* must equal T */
+  const int64_t* target;    /* [T] replayed token y, 0 <= y < V */
+  const float* temperature; /* [T] finite, > 0 */
+  const int32_t* top_k;     /* [T] <= 0 or >= V: off */
+  const float* top_p;       /* [T] in (0, 1]; 1.0: exact identity */
+  const float* min_p;       /* [T] in [0, 1]; 0: off */
+} sts_rows;
+
+/* Per-row scalars written by the forward and read by the backward (the only
+ * state kept between them: item 2, "saving only per-row scalars"). */
+typedef struct {
+  float* row_max;        /* [T] max_i s_i over the unfiltered row */
+  float* lse_support;    /* [T] log sum_{i in S} exp(s_i) */
+  float* cut_logit;      /* [T] s of the last kept token in (s desc, id asc) */
+  int32_t* cut_id;       /* [T] id  of the last kept token */
+  int32_t* support_size; /* [T] |S| */
+  int32_t* flags;        /* [T] STS_ROW_* bits */
+} sts_saved;
+
+#define STS_ROW_TARGET_IN_SUPPORT 1 /* y in S */
+#define STS_ROW_INVALID 2           /* row failed validation */
+#define STS_ROW_IDENTITY 4          /* no active filter */
+
+/* Bytes of workspace needed. pass: 0 forward (also sts_sample), 1 backward,
+ * 2 sts_filter_logits. Returns 0 for an invalid shape. */
+size_t sts_workspace_bytes(const sts_shape* shape, int pass);
+
+/* Forward: logprob[T] (fp32) and the saved per-row scalars.
+ * ws must hold sts_workspace_bytes(shape, 0) bytes. */
+sts_status sts_forward(const sts_shape* shape, const void* H_bf16, const void* W_bf16,
+                       const sts_rows* rows, float* logprob, const sts_saved* saved,
+                       void* ws, size_t ws_bytes, sts_stream_t stream);
+
+/* Backward: dH[T,d] and dW[V,d] (fp32) from grad_logprob[T] and the scalars
+ * saved by sts_forward on the same H, W and rows. dH is overwritten; dW is
+ * overwritten unless accumulate_dW is non-zero (then dW += result).
+ * ws must hold sts_workspace_bytes(shape, 1) bytes. */
+sts_status sts_backward(const sts_shape* shape, const void* H_bf16, const void* W_bf16,
+                        const sts_rows* rows, const sts_saved* saved,
+                        const float* grad_logprob, float* dH, float* dW, int accumulate_dW,
+                        void* ws, size_t ws_bytes, sts_stream_t stream);
+
+/* Draw one token per row from the filtered distribution: the inverse CDF of
+ * the support walked in (s desc, id asc) order, taking the first kept token
+ * whose inclusive running mass exceeds u[t] * sum_{i in S} exp(s_i - m).
+ * rows->target is ignored (may be NULL). u: [T] doubles in [0, 1).
+ * ws: sts_workspace_bytes(shape, 0). Used to replay rollouts for tests and
+ * benchmarks; the pages fix no sampler, only the support it draws from. */
+sts_status sts_sample(const sts_shape* shape, const void* H_bf16, const void* W_bf16,
+                      const sts_rows* rows, const double* u, int64_t* sampled,
+                      void* ws, size_t ws_bytes, sts_stream_t stream);
+
+/* Test hook: run only the support program on caller-given fp32 scaled logits
+ * [T, V] (row stride V). Writes support_size, cut_logit, cut_id per row and,
+ * when mask is not NULL, mask[T, V] (1 = kept). rows->target is ignored.
+ * ws: sts_workspace_bytes(shape, 2). */
+sts_status sts_filter_logits(const sts_shape* shape, const float* scaled_logits,
+                             const sts_rows* rows, int32_t* support_size, float* cut_logit,
+                             int32_t* cut_id, uint8_t* mask, void* ws, size_t ws_bytes,
+                             sts_stream_t stream);
+
+/* Test hook: the forward's first pass alone, S[t, v] = (H . W^T)[t, v] /
+ * temperature[t] for t in [t0, t0 + rows), v in [v0, v0 + cols), written to
+ * S_out[(t - t0) * ld + (v - v0)] (fp32). t0 must be a multiple of 128 and v0
+ * of 256 (the tile grid of the forward); ld a multiple of 4, >= cols.
+ * Allocates nothing; a device-side wait timeout in this hook is not reported. */
+sts_status sts_scaled_logits(const sts_shape* shape, const void* H_bf16, const void* W_bf16,
+                             const float* temperature, int64_t t0, int64_t rows, int64_t v0,
+                             int64_t cols, float* S_out, int64_t ld, sts_stream_t stream);
+
+/* Synchronise the stream and read the status word a previous call left in
+ * ws. first_bad_row (may be NULL) receives the lowest failing row or -1. */
+sts_status sts_get_status(const void* ws, sts_stream_t stream, int64_t* first_bad_row);
+
+const char* sts_status_string(sts_status status);
+
+int sts_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STS_H_ */

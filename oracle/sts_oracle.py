@@ -91,19 +91,24 @@ class RowFilter:
         return int(self.order[self.size - 1])
 
 
-def scaled_logits(H, W, temperature) -> np.ndarray:
+def scaled_logits(H, W, temperature, vocab_slice=None) -> np.ndarray:
     """s = (H . W^T) / tau in float64.
 
     [xorl#74] "What this PR does", item 2 (chunked projection, fp32-output GEMM
     on the generic lane) and "Self-review pass" (per-row temperature applied
     after the GEMM). The oracle keeps the full float64 product of the bf16
     operand values, which is the exact logit up to one float64 rounding per
-    accumulation step.
+    accumulation step. ``vocab_slice`` only bounds host memory: W is widened
+    to float64 that many rows at a time; every logit is the same dot product.
     """
     H = np.asarray(H, dtype=np.float64)
-    W = np.asarray(W, dtype=np.float64)
     tau = np.asarray(temperature, dtype=np.float64)
-    return (H @ W.T) / tau[:, None]
+    V = W.shape[0]
+    step = V if vocab_slice is None else int(vocab_slice)
+    z = np.empty((H.shape[0], V), dtype=np.float64)
+    for a in range(0, V, step):
+        z[:, a:a + step] = H @ np.asarray(W[a:a + step], dtype=np.float64).T
+    return z / tau[:, None]
 
 
 def filter_row(s, top_k: int, top_p: float, min_p: float) -> RowFilter:
@@ -266,20 +271,24 @@ def logit_grad(s, rows, grad_logprob):
     return dZ
 
 
-def backward(H, W, rows, grad_logprob, s=None, vocab_rows=None):
+def backward(H, W, rows, grad_logprob, s=None, vocab_rows=None, vocab_slice=None):
     """Closed-form VJP: dH = dZ . W and dW = dZ^T . H in float64.
 
     [xorl#74] item 2 (recompute closed-form VJP) and "Acceptance criteria"
     (hidden and weight gradients). ``vocab_rows`` restricts dW to the listed
     vocabulary rows (the full [V, d] float64 matrix of the large workloads
-    does not fit comfortably in host memory).
+    does not fit comfortably in host memory); ``vocab_slice`` widens W to
+    float64 that many rows at a time for dH = sum over vocabulary slices.
     """
     H = np.asarray(H, dtype=np.float64)
-    W = np.asarray(W, dtype=np.float64)
     if s is None:
-        s = scaled_logits(H, W, rows["temperature"])
+        s = scaled_logits(H, W, rows["temperature"], vocab_slice=vocab_slice)
     dZ = logit_grad(s, rows, grad_logprob)
-    dH = dZ @ W
+    V = W.shape[0]
+    step = V if vocab_slice is None else int(vocab_slice)
+    dH = np.zeros((H.shape[0], H.shape[1]), dtype=np.float64)
+    for a in range(0, V, step):
+        dH += dZ[:, a:a + step] @ np.asarray(W[a:a + step], dtype=np.float64)
     if vocab_rows is None:
         dW = dZ.T @ H
     else:

@@ -1,0 +1,343 @@
+"""B200 (sm_100a) sampling-transform scoring core: thin Python binding.
+
+Each function marshals torch tensors into the C ABI of ``libsts.so``
+(declared in ``include/sts.h``) and calls the entry point of the same name.
+Every step of the computation runs in the library's CUDA kernels; there is
+no Python or CPU fallback, and a missing library raises ``StsError``.
+
+The operation ("Consolidate sampling-transform scoring on one shared chunked
+core; implement top-k/top-p/min-p replay for generic ce_modes", xorl PR 74,
+"What this PR does", items 1, 2 and 4): per row, logits z = H . W^T with fp32
+accumulation, s = z / temperature, the support program top-k -> top-p ->
+min-p with token-id tie-break, and the selected token's logprob on the
+filtered support; the backward recomputes the logits and forms
+dz = g (onehot - p_support) / temperature inside the GEMM epilogue.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "StsError",
+    "load",
+    "library_path",
+    "sts_workspace_bytes",
+    "sts_forward",
+    "sts_backward",
+    "sts_sample",
+    "sts_filter_logits",
+    "sts_scaled_logits",
+    "sts_get_status",
+    "sts_status_string",
+    "ROW_TARGET_IN_SUPPORT",
+    "ROW_INVALID",
+    "ROW_IDENTITY",
+    "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libsts.so")
+
+STS_OK = 0
+STS_ERR_NULL = 1
+STS_ERR_SHAPE = 2
+STS_ERR_DTYPE = 3
+STS_ERR_WORKSPACE = 9
+ROW_TARGET_IN_SUPPORT = 1
+ROW_INVALID = 2
+ROW_IDENTITY = 4
+
+EXPORTED_SYMBOLS = (
+    "sts_workspace_bytes",
+    "sts_forward",
+    "sts_backward",
+    "sts_sample",
+    "sts_filter_logits",
+    "sts_scaled_logits",
+    "sts_get_status",
+    "sts_status_string",
+    "sts_abi_version",
+)
+
+
+class StsError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        msg = _status_text(self.status)
+        super().__init__(f"{what}: {msg} (status {self.status})" if what else msg)
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("V", ctypes.c_int64),
+                ("vocab_chunk", ctypes.c_int64), ("row_chunk", ctypes.c_int64)]
+
+
+class _Rows(ctypes.Structure):
+    _fields_ = [("len", ctypes.c_int64), ("target", ctypes.c_void_p),
+                ("temperature", ctypes.c_void_p), ("top_k", ctypes.c_void_p),
+                ("top_p", ctypes.c_void_p), ("min_p", ctypes.c_void_p)]
+
+
+class _Saved(ctypes.Structure):
+    _fields_ = [("row_max", ctypes.c_void_p), ("lse_support", ctypes.c_void_p),
+                ("cut_logit", ctypes.c_void_p), ("cut_id", ctypes.c_void_p),
+                ("support_size", ctypes.c_void_p), ("flags", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load ``libsts.so`` (raises StsError / OSError when it is absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise OSError(f"{_LIB_PATH} is missing: build it with "
+                      "`python -m sampling_transform_lm_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, S, I64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64
+    lib.sts_workspace_bytes.argtypes = [ctypes.POINTER(_Shape), ctypes.c_int]
+    lib.sts_workspace_bytes.restype = S
+    lib.sts_forward.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows), P,
+                                ctypes.POINTER(_Saved), P, S, P]
+    lib.sts_forward.restype = ctypes.c_int
+    lib.sts_backward.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows),
+                                 ctypes.POINTER(_Saved), P, P, P, ctypes.c_int, P, S, P]
+    lib.sts_backward.restype = ctypes.c_int
+    lib.sts_sample.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows), P, P, P, S, P]
+    lib.sts_sample.restype = ctypes.c_int
+    lib.sts_filter_logits.argtypes = [ctypes.POINTER(_Shape), P, ctypes.POINTER(_Rows), P, P, P, P,
+                                      P, S, P]
+    lib.sts_filter_logits.restype = ctypes.c_int
+    lib.sts_scaled_logits.argtypes = [ctypes.POINTER(_Shape), P, P, P, I64, I64, I64, I64, P, I64, P]
+    lib.sts_scaled_logits.restype = ctypes.c_int
+    lib.sts_get_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
+    lib.sts_get_status.restype = ctypes.c_int
+    lib.sts_status_string.argtypes = [ctypes.c_int]
+    lib.sts_status_string.restype = ctypes.c_char_p
+    lib.sts_abi_version.argtypes = []
+    lib.sts_abi_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _status_text(status: int) -> str:
+    try:
+        return load().sts_status_string(int(status)).decode()
+    except OSError:
+        return f"status {status}"
+
+
+def sts_status_string(status: int) -> str:
+    return _status_text(status)
+
+
+def _check(status: int, what: str):
+    if status != STS_OK:
+        raise StsError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _shape(T, d, V, vocab_chunk=0, row_chunk=0):
+    return _Shape(int(T), int(d), int(V), int(vocab_chunk), int(row_chunk))
+
+
+def _need(t, dtype, name, shape=None):
+    if t.dtype != dtype:
+        status = STS_ERR_DTYPE if dtype == torch.bfloat16 else STS_ERR_SHAPE
+        raise StsError(status, f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise StsError(STS_ERR_SHAPE, f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise StsError(STS_ERR_SHAPE, f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise StsError(STS_ERR_SHAPE, f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _rows(T, target, temperature, top_k, top_p, min_p):
+    for name, t, dt in (("temperature", temperature, torch.float32), ("top_k", top_k, torch.int32),
+                        ("top_p", top_p, torch.float32), ("min_p", min_p, torch.float32)):
+        _need(t, dt, name)
+        if t.dim() != 1:
+            raise StsError(STS_ERR_SHAPE, f"{name} must be 1-D")
+        if t.shape[0] != T:  # over- or under-length metadata is rejected, never truncated
+            raise StsError(STS_ERR_SHAPE, f"{name} has {t.shape[0]} rows, expected {T}")
+    if target is not None:
+        _need(target, torch.int64, "target", (T,))
+    return _Rows(T, _ptr(target), _ptr(temperature), _ptr(top_k), _ptr(top_p), _ptr(min_p))
+
+
+def sts_workspace_bytes(T, d, V, pass_, vocab_chunk=0, row_chunk=0) -> int:
+    sh = _shape(T, d, V, vocab_chunk, row_chunk)
+    n = load().sts_workspace_bytes(ctypes.byref(sh), int(pass_))
+    if n == 0:
+        raise StsError(STS_ERR_SHAPE, "sts_workspace_bytes")
+    return int(n)
+
+
+def _workspace(nbytes, device, ws=None):
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise StsError(STS_ERR_WORKSPACE, f"workspace holds {ws.numel()} bytes, needs {nbytes}")
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _hw(H, W):
+    for name, t in (("H", H), ("W", W)):  # dtype first: an fp8 head is a dtype error
+        if t.dtype != torch.bfloat16:
+            raise StsError(STS_ERR_DTYPE, f"{name} must be torch.bfloat16, got {t.dtype}")
+    _need(H, torch.bfloat16, "H")
+    _need(W, torch.bfloat16, "W")
+    if H.dim() != 2 or W.dim() != 2 or H.shape[1] != W.shape[1]:
+        raise StsError(STS_ERR_SHAPE, "H must be [T, d] and W [V, d]")
+    return H.shape[0], H.shape[1], W.shape[0]
+
+
+def sts_forward(H, W, target, temperature, top_k, top_p, min_p, *, row_chunk=0, ws=None,
+                stream=None, check=False):
+    """Filtered-support logprob per row plus the saved per-row scalars.
+
+    Returns ``(logprob [T] fp32, saved dict, workspace)``. With ``check`` the
+    call synchronises and raises on a row-value error.
+    """
+    lib = load()
+    T, d, V = _hw(H, W)
+    rows = _rows(T, target, temperature, top_k, top_p, min_p)
+    sh = _shape(T, d, V, 0, row_chunk)
+    dev = H.device
+    ws = _workspace(sts_workspace_bytes(T, d, V, 0, 0, row_chunk), dev, ws)
+    logprob = torch.empty(T, dtype=torch.float32, device=dev)
+    saved = {
+        "row_max": torch.empty(T, dtype=torch.float32, device=dev),
+        "lse_support": torch.empty(T, dtype=torch.float32, device=dev),
+        "cut_logit": torch.empty(T, dtype=torch.float32, device=dev),
+        "cut_id": torch.empty(T, dtype=torch.int32, device=dev),
+        "support_size": torch.empty(T, dtype=torch.int32, device=dev),
+        "flags": torch.empty(T, dtype=torch.int32, device=dev),
+    }
+    sv = _Saved(*(_ptr(saved[k]) for k in ("row_max", "lse_support", "cut_logit", "cut_id",
+                                            "support_size", "flags")))
+    st = lib.sts_forward(ctypes.byref(sh), _ptr(H), _ptr(W), ctypes.byref(rows), _ptr(logprob),
+                         ctypes.byref(sv), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "sts_forward")
+    if check:
+        sts_get_status(ws, stream, raise_on_error=True)
+    return logprob, saved, ws
+
+
+def sts_backward(H, W, target, temperature, top_k, top_p, min_p, saved, grad_logprob, *,
+                 dW=None, accumulate_dW=False, vocab_chunk=0, ws=None, stream=None, check=False):
+    """dH [T, d] and dW [V, d] (fp32) of sum_t g_t * logprob_t."""
+    lib = load()
+    T, d, V = _hw(H, W)
+    rows = _rows(T, target, temperature, top_k, top_p, min_p)
+    _need(grad_logprob, torch.float32, "grad_logprob", (T,))
+    sh = _shape(T, d, V, vocab_chunk, 0)
+    dev = H.device
+    ws = _workspace(sts_workspace_bytes(T, d, V, 1, vocab_chunk, 0), dev, ws)
+    dH = torch.empty((T, d), dtype=torch.float32, device=dev)
+    if dW is None:
+        if accumulate_dW:
+            raise StsError(STS_ERR_NULL, "accumulate_dW needs a dW tensor")
+        dW = torch.empty((V, d), dtype=torch.float32, device=dev)
+    else:
+        _need(dW, torch.float32, "dW", (V, d))
+    sv = _Saved(*(_ptr(saved[k]) for k in ("row_max", "lse_support", "cut_logit", "cut_id",
+                                            "support_size", "flags")))
+    st = lib.sts_backward(ctypes.byref(sh), _ptr(H), _ptr(W), ctypes.byref(rows), ctypes.byref(sv),
+                          _ptr(grad_logprob), _ptr(dH), _ptr(dW), 1 if accumulate_dW else 0,
+                          _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "sts_backward")
+    if check:
+        sts_get_status(ws, stream, raise_on_error=True)
+    return dH, dW
+
+
+def sts_sample(H, W, temperature, top_k, top_p, min_p, u, *, row_chunk=0, ws=None, stream=None,
+               check=False):
+    """One token per row drawn from the filtered distribution with uniforms u."""
+    lib = load()
+    T, d, V = _hw(H, W)
+    rows = _rows(T, None, temperature, top_k, top_p, min_p)
+    _need(u, torch.float64, "u", (T,))
+    sh = _shape(T, d, V, 0, row_chunk)
+    ws = _workspace(sts_workspace_bytes(T, d, V, 0, 0, row_chunk), H.device, ws)
+    out = torch.empty(T, dtype=torch.int64, device=H.device)
+    st = lib.sts_sample(ctypes.byref(sh), _ptr(H), _ptr(W), ctypes.byref(rows), _ptr(u), _ptr(out),
+                        _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "sts_sample")
+    if check:
+        sts_get_status(ws, stream, raise_on_error=True)
+    return out
+
+
+def sts_filter_logits(S, top_k, top_p, min_p, *, want_mask=False, ws=None, stream=None, check=False):
+    """The support program alone on fp32 scaled logits S [T, V]."""
+    lib = load()
+    _need(S, torch.float32, "S")
+    T, V = S.shape
+    for name, t, dt in (("top_k", top_k, torch.int32), ("top_p", top_p, torch.float32),
+                        ("min_p", min_p, torch.float32)):
+        _need(t, dt, name, (T,))
+    rows = _Rows(T, None, None, _ptr(top_k), _ptr(top_p), _ptr(min_p))
+    sh = _shape(T, 8, V)
+    ws = _workspace(sts_workspace_bytes(T, 8, V, 2), S.device, ws)
+    size = torch.empty(T, dtype=torch.int32, device=S.device)
+    cut_logit = torch.empty(T, dtype=torch.float32, device=S.device)
+    cut_id = torch.empty(T, dtype=torch.int32, device=S.device)
+    mask = torch.empty((T, V), dtype=torch.uint8, device=S.device) if want_mask else None
+    st = lib.sts_filter_logits(ctypes.byref(sh), _ptr(S), ctypes.byref(rows), _ptr(size),
+                               _ptr(cut_logit), _ptr(cut_id), _ptr(mask), _ptr(ws), ws.numel(),
+                               _stream(stream))
+    _check(st, "sts_filter_logits")
+    if check:
+        sts_get_status(ws, stream, raise_on_error=True)
+    return {"size": size, "cut_logit": cut_logit, "cut_id": cut_id, "mask": mask}
+
+
+def sts_scaled_logits(H, W, temperature, t0=0, rows=None, v0=0, cols=None, *, out=None,
+                      stream=None):
+    """The forward's first pass alone: S = (H . W^T) / temperature (fp32)."""
+    lib = load()
+    T, d, V = _hw(H, W)
+    _need(temperature, torch.float32, "temperature", (T,))
+    rows = T - t0 if rows is None else rows
+    cols = V - v0 if cols is None else cols
+    ld = (cols + 3) // 4 * 4
+    if out is None:
+        out = torch.empty((rows, ld), dtype=torch.float32, device=H.device)
+    sh = _shape(T, d, V)
+    st = lib.sts_scaled_logits(ctypes.byref(sh), _ptr(H), _ptr(W), _ptr(temperature), int(t0),
+                               int(rows), int(v0), int(cols), _ptr(out), int(out.stride(0)),
+                               _stream(stream))
+    _check(st, "sts_scaled_logits")
+    return out[:, :cols]
+
+
+def sts_get_status(ws, stream=None, raise_on_error=False):
+    """Synchronise and read the status word left in ``ws``: (status, first_bad_row)."""
+    lib = load()
+    row = ctypes.c_int64(-1)
+    st = lib.sts_get_status(_ptr(ws), _stream(stream), ctypes.byref(row))
+    if raise_on_error and st != STS_OK:
+        raise StsError(st, f"row {row.value}" if row.value >= 0 else "device status")
+    return int(st), int(row.value)

@@ -1,0 +1,504 @@
+// C ABI of the scoring core: argument checks, workspace carving, tensor maps
+// and the launch sequence of the forward / backward / sample / filter paths.
+//
+//   forward   validate rows -> per row chunk: [tcgen05 GEMM, epilogue s = z/tau
+//             -> fp32 chunk of scaled logits] -> [exact per-row resolver]
+//   backward  per vocabulary chunk: [recompute GEMM with the dz epilogue ->
+//             bf16 dZ chunk] -> [dW slice GEMM, written once] -> [dH GEMM,
+//             stored for the first chunk, TMA reduce-added after]
+//
+// ("Consolidate sampling-transform scoring on one shared chunked core", xorl
+// PR 74: "What this PR does", item 2, chunked core with a recompute VJP; the
+// "Self-review pass" single-pass vocabulary-chunked backward with write-once
+// weight-gradient slices.)
+#include <cstring>
+#include <mutex>
+
+#include "gemm_sm100.cuh"
+#include "sts_internal.h"
+
+namespace sts {
+namespace {
+
+constexpr int64_t kDefaultVocabChunk = 16384;
+constexpr size_t kDefaultChunkBytes = size_t(4) << 30;  // forward logits chunk budget
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool map2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+           uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  std::memset(m, 0, sizeof(*m));
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 operand, K contiguous: [rows][K] with row stride ld elements.
+bool map_kmajor(CUtensorMap* m, const void* p, int64_t K, int64_t rows, int64_t ld, uint32_t box_rows) {
+  return map2d(m, p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)K, (uint64_t)rows, (uint64_t)ld * 2,
+               64, box_rows);
+}
+
+// bf16 operand, MN contiguous: [K][MN] with row stride ld elements.
+bool map_mnmajor(CUtensorMap* m, const void* p, int64_t MN, int64_t K, int64_t ld) {
+  return map2d(m, p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)MN, (uint64_t)K, (uint64_t)ld * 2,
+               64, 64);
+}
+
+bool map_out_f32(CUtensorMap* m, const void* p, int64_t cols, int64_t rows, int64_t ld) {
+  return map2d(m, p, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)cols, (uint64_t)rows,
+               (uint64_t)ld * 4, 32, 32);
+}
+
+bool map_out_bf16(CUtensorMap* m, const void* p, int64_t cols, int64_t rows, int64_t ld) {
+  return map2d(m, p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)cols, (uint64_t)rows,
+               (uint64_t)ld * 2, 64, 32);
+}
+
+template <bool AMN, bool BMN, int EPI>
+cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
+                     const GemmParams& p, int sms, cudaStream_t st) {
+  auto kern = gemm_kernel<AMN, BMN, EPI>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMM_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const long long tiles =
+      (long long)((p.M + GEMM_BM - 1) / GEMM_BM) * (long long)((p.N + GEMM_BN - 1) / GEMM_BN);
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(a, b, c, p);
+  return cudaGetLastError();
+}
+
+struct DeviceInfo {
+  bool ok;
+  int sms;
+};
+
+sts_status device_info(DeviceInfo& info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return STS_ERR_CUDA;
+  static DeviceInfo cache[64];
+  static bool have[64];
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return STS_ERR_CUDA;
+  if (!have[dev]) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return STS_ERR_CUDA;
+    cache[dev].ok = (prop.major == 10 && prop.minor == 0);
+    cache[dev].sms = prop.multiProcessorCount;
+    have[dev] = true;
+  }
+  info = cache[dev];
+  return info.ok ? STS_OK : STS_ERR_UNSUPPORTED_ARCH;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- shapes
+
+bool shape_ok(const sts_shape* s) {
+  if (!s) return false;
+  if (s->T < 1 || s->T > (int64_t(1) << 31) - 1) return false;
+  if (s->V < 1 || s->V > (int64_t(1) << 31) - 1) return false;
+  if (s->d < 8 || (s->d % 8) != 0 || s->d > (int64_t(1) << 20)) return false;
+  if (s->vocab_chunk < 0 || (s->vocab_chunk % 256) != 0) return false;
+  if (s->row_chunk < 0 || (s->row_chunk % 128) != 0) return false;
+  return true;
+}
+
+int64_t logits_ld(const sts_shape* s) { return (s->V + 3) / 4 * 4; }
+
+int64_t row_chunk(const sts_shape* s) {
+  const int64_t Tpad = (s->T + 127) / 128 * 128;
+  int64_t rc = s->row_chunk;
+  if (rc == 0) {
+    const int64_t per_row = logits_ld(s) * 4;
+    rc = (int64_t)(kDefaultChunkBytes / (size_t)per_row) / 128 * 128;
+    if (rc < 128) rc = 128;
+  }
+  return rc < Tpad ? rc : Tpad;
+}
+
+int64_t vocab_chunk(const sts_shape* s) {
+  const int64_t Vpad = (s->V + 255) / 256 * 256;
+  const int64_t vc = s->vocab_chunk ? s->vocab_chunk : kDefaultVocabChunk;
+  return vc < Vpad ? vc : Vpad;
+}
+
+struct FwdLayout {
+  size_t flags_off, logits_off, total;
+};
+
+FwdLayout fwd_layout(const sts_shape* s) {
+  FwdLayout L;
+  L.flags_off = sizeof(WsHeader);
+  L.logits_off = align_up(L.flags_off + (size_t)s->T * 4, kAlign);
+  L.total = align_up(L.logits_off + (size_t)row_chunk(s) * (size_t)logits_ld(s) * 4, kAlign);
+  return L;
+}
+
+struct BwdLayout {
+  size_t dz_off, total;
+};
+
+BwdLayout bwd_layout(const sts_shape* s) {
+  BwdLayout L;
+  L.dz_off = kAlign;
+  L.total = align_up(L.dz_off + (size_t)s->T * (size_t)vocab_chunk(s) * 2, kAlign);
+  return L;
+}
+
+size_t filter_bytes(const sts_shape* s) { return align_up(sizeof(WsHeader) + (size_t)s->T * 4, kAlign); }
+
+sts_status check_rows(const sts_shape* s, const sts_rows* r, bool need_target) {
+  if (!r) return STS_ERR_NULL;
+  if (r->len != s->T) return STS_ERR_SHAPE;
+  if (!r->temperature || !r->top_k || !r->top_p || !r->min_p) return STS_ERR_NULL;
+  if (need_target && !r->target) return STS_ERR_NULL;
+  return STS_OK;
+}
+
+sts_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return STS_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return STS_ERR_WORKSPACE;
+  if (ws_bytes < need) return STS_ERR_WORKSPACE;
+  return STS_OK;
+}
+
+sts_status reset_header(void* ws, cudaStream_t st) {
+  WsHeader* h = static_cast<WsHeader*>(ws);
+  if (cudaMemsetAsync(&h->bad_row_code, 0xFF, sizeof(h->bad_row_code), st) != cudaSuccess)
+    return STS_ERR_CUDA;
+  if (cudaMemsetAsync(&h->err, 0, sizeof(h->err), st) != cudaSuccess) return STS_ERR_CUDA;
+  return STS_OK;
+}
+
+#define STS_TRY(x)                     \
+  do {                                 \
+    const sts_status _s = (x);         \
+    if (_s != STS_OK) return _s;       \
+  } while (0)
+
+#define STS_CUDA(x)                                    \
+  do {                                                 \
+    if ((x) != cudaSuccess) return STS_ERR_CUDA;       \
+  } while (0)
+
+// Forward-style pass shared by sts_forward and sts_sample.
+sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, const sts_rows* rows,
+                        float* logprob, const sts_saved* saved, const double* u, int64_t* sampled,
+                        void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!shape_ok(shape)) return STS_ERR_SHAPE;
+  if (!H || !W) return STS_ERR_NULL;
+  const bool fwd = (sampled == nullptr);
+  STS_TRY(check_rows(shape, rows, fwd));
+  if (fwd) {
+    if (!logprob || !saved || !saved->row_max || !saved->lse_support || !saved->cut_logit ||
+        !saved->cut_id || !saved->support_size || !saved->flags)
+      return STS_ERR_NULL;
+  } else if (!u) {
+    return STS_ERR_NULL;
+  }
+  if (!aligned16(H) || !aligned16(W)) return STS_ERR_SHAPE;
+  const FwdLayout L = fwd_layout(shape);
+  STS_TRY(check_ws(ws, ws_bytes, L.total));
+  DeviceInfo dev;
+  STS_TRY(device_info(dev));
+
+  const int64_t T = shape->T, V = shape->V, d = shape->d;
+  const int64_t ld = logits_ld(shape), rc_max = row_chunk(shape);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+  int32_t* flags = fwd ? saved->flags : reinterpret_cast<int32_t*>(wsb + L.flags_off);
+  float* S = reinterpret_cast<float*>(wsb + L.logits_off);
+
+  STS_TRY(reset_header(ws, st));
+  launch_validate(rows->target, rows->temperature, rows->top_p, rows->min_p, T, V, flags, hdr, fwd, st);
+  STS_CUDA(cudaGetLastError());
+
+  CUtensorMap ma, mb;
+  if (!map_kmajor(&ma, H, d, T, d, GEMM_BM) || !map_kmajor(&mb, W, d, V, d, GEMM_BN))
+    return STS_ERR_CUDA;
+
+  for (int64_t t0 = 0; t0 < T; t0 += rc_max) {
+    const int64_t rc = (T - t0) < rc_max ? (T - t0) : rc_max;
+    CUtensorMap mc;
+    if (!map_out_f32(&mc, S, V, rc, ld)) return STS_ERR_CUDA;
+    GemmParams p{};
+    p.M = (int)rc;
+    p.N = (int)V;
+    p.K = (int)d;
+    p.a_mn0 = (int)t0;
+    p.tau = rows->temperature + t0;
+    p.err = &hdr->err;
+    STS_CUDA((run_gemm<false, false, kEpiLogits>(ma, mb, mc, p, dev.sms, st)));
+
+    ResolveArgs a{};
+    a.S = S;
+    a.ld = ld;
+    a.rows = (int)rc;
+    a.V = (int)V;
+    a.mode = fwd ? kModeForward : kModeSample;
+    a.target = fwd ? rows->target + t0 : nullptr;
+    a.top_k = rows->top_k + t0;
+    a.top_p = rows->top_p + t0;
+    a.min_p = rows->min_p + t0;
+    a.u = fwd ? nullptr : u + t0;
+    a.row_flags = flags + t0;
+    a.flags_out = flags + t0;
+    if (fwd) {
+      a.logprob = logprob + t0;
+      a.row_max = saved->row_max + t0;
+      a.lse_support = saved->lse_support + t0;
+      a.cut_logit = saved->cut_logit + t0;
+      a.cut_id = saved->cut_id + t0;
+      a.support_size = saved->support_size + t0;
+    } else {
+      a.sampled = sampled + t0;
+    }
+    a.hdr = hdr;
+    a.row_base = t0;
+    STS_CUDA(launch_resolve(a, dev.sms, st));
+  }
+  return STS_OK;
+}
+
+}  // namespace
+}  // namespace sts
+
+using namespace sts;
+
+extern "C" {
+
+int sts_abi_version(void) { return STS_ABI_VERSION; }
+
+const char* sts_status_string(sts_status s) {
+  switch (s) {
+    case STS_OK: return "ok";
+    case STS_ERR_NULL: return "a required pointer is NULL";
+    case STS_ERR_SHAPE: return "invalid shape, alignment or metadata length";
+    case STS_ERR_DTYPE: return "operands must be bf16 (fp8 heads are not supported)";
+    case STS_ERR_TEMPERATURE: return "temperature must be finite and > 0";
+    case STS_ERR_TOP_K: return "invalid top_k";
+    case STS_ERR_TOP_P: return "top_p must be in (0, 1]";
+    case STS_ERR_MIN_P: return "min_p must be in [0, 1]";
+    case STS_ERR_TARGET: return "target must be in [0, V)";
+    case STS_ERR_WORKSPACE: return "workspace missing, misaligned (256 B) or too small";
+    case STS_ERR_OVERFLOW: return "an internal bound was exceeded";
+    case STS_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case STS_ERR_CUDA: return "a CUDA call failed";
+    case STS_ERR_UNSUPPORTED_ARCH: return "device is not sm_100 (B200)";
+  }
+  return "unknown status";
+}
+
+size_t sts_workspace_bytes(const sts_shape* shape, int pass) {
+  if (!shape_ok(shape)) return 0;
+  switch (pass) {
+    case 0: return fwd_layout(shape).total;
+    case 1: return bwd_layout(shape).total;
+    case 2: return filter_bytes(shape);
+  }
+  return 0;
+}
+
+sts_status sts_forward(const sts_shape* shape, const void* H, const void* W, const sts_rows* rows,
+                       float* logprob, const sts_saved* saved, void* ws, size_t ws_bytes,
+                       sts_stream_t stream) {
+  return forward_impl(shape, H, W, rows, logprob, saved, nullptr, nullptr, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+sts_status sts_sample(const sts_shape* shape, const void* H, const void* W, const sts_rows* rows,
+                      const double* u, int64_t* sampled, void* ws, size_t ws_bytes,
+                      sts_stream_t stream) {
+  if (!sampled) return STS_ERR_NULL;
+  return forward_impl(shape, H, W, rows, nullptr, nullptr, u, sampled, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, const sts_rows* rows,
+                        const sts_saved* saved, const float* grad, float* dH, float* dW,
+                        int accumulate_dW, void* ws, size_t ws_bytes, sts_stream_t stream) {
+  if (!shape_ok(shape)) return STS_ERR_SHAPE;
+  if (!H || !W || !grad || !dH || !dW) return STS_ERR_NULL;
+  STS_TRY(check_rows(shape, rows, true));
+  if (!saved || !saved->lse_support || !saved->cut_logit || !saved->cut_id || !saved->flags)
+    return STS_ERR_NULL;
+  if (!aligned16(H) || !aligned16(W) || !aligned16(dH) || !aligned16(dW)) return STS_ERR_SHAPE;
+  const BwdLayout L = bwd_layout(shape);
+  STS_TRY(check_ws(ws, ws_bytes, L.total));
+  DeviceInfo dev;
+  STS_TRY(device_info(dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  const int64_t T = shape->T, V = shape->V, d = shape->d, Vc = vocab_chunk(shape);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+  void* dZ = wsb + L.dz_off;
+  STS_TRY(reset_header(ws, st));
+
+  CUtensorMap m_h_k, m_w_k, m_h_mn, m_w_mn, m_dw, m_dh;
+  if (!map_kmajor(&m_h_k, H, d, T, d, GEMM_BM) || !map_kmajor(&m_w_k, W, d, V, d, GEMM_BN) ||
+      !map_mnmajor(&m_h_mn, H, d, T, d) || !map_mnmajor(&m_w_mn, W, d, V, d) ||
+      !map_out_f32(&m_dw, dW, d, V, d) || !map_out_f32(&m_dh, dH, d, T, d))
+    return STS_ERR_CUDA;
+
+  for (int64_t v0 = 0; v0 < V; v0 += Vc) {
+    const int64_t w = (V - v0) < Vc ? (V - v0) : Vc;
+    CUtensorMap m_dz_out, m_dz_k, m_dz_mn;
+    if (!map_out_bf16(&m_dz_out, dZ, w, T, Vc) || !map_kmajor(&m_dz_k, dZ, w, T, Vc, GEMM_BM) ||
+        !map_mnmajor(&m_dz_mn, dZ, w, T, Vc))
+      return STS_ERR_CUDA;
+
+    // 1. recompute the chunk's logits and form dZ in the epilogue
+    GemmParams p{};
+    p.M = (int)T;
+    p.N = (int)w;
+    p.K = (int)d;
+    p.b_mn0 = (int)v0;
+    p.tau = rows->temperature;
+    p.lse = saved->lse_support;
+    p.cut_logit = saved->cut_logit;
+    p.cut_id = saved->cut_id;
+    p.target = rows->target;
+    p.grad = grad;
+    p.flags = saved->flags;
+    p.col_base = (int)v0;
+    p.err = &hdr->err;
+    STS_CUDA((run_gemm<false, false, kEpiDZ>(m_h_k, m_w_k, m_dz_out, p, dev.sms, st)));
+
+    // 2. dW[v0:v0+w] = dZ^T . H (both operands MN-major), written once
+    GemmParams q{};
+    q.M = (int)w;
+    q.N = (int)d;
+    q.K = (int)T;
+    q.c_y0 = (int)v0;
+    q.err = &hdr->err;
+    if (accumulate_dW)
+      STS_CUDA((run_gemm<true, true, kEpiReduceF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st)));
+    else
+      STS_CUDA((run_gemm<true, true, kEpiStoreF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st)));
+
+    // 3. dH (+)= dZ . W[v0:v0+w] (W read MN-major)
+    GemmParams r{};
+    r.M = (int)T;
+    r.N = (int)d;
+    r.K = (int)w;
+    r.b_k0 = (int)v0;
+    r.err = &hdr->err;
+    if (v0 == 0)
+      STS_CUDA((run_gemm<false, true, kEpiStoreF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st)));
+    else
+      STS_CUDA((run_gemm<false, true, kEpiReduceF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st)));
+  }
+  return STS_OK;
+}
+
+sts_status sts_filter_logits(const sts_shape* shape, const float* S, const sts_rows* rows,
+                             int32_t* support_size, float* cut_logit, int32_t* cut_id,
+                             uint8_t* mask, void* ws, size_t ws_bytes, sts_stream_t stream) {
+  if (!shape_ok(shape)) return STS_ERR_SHAPE;
+  if (!S || !support_size || !cut_logit || !cut_id) return STS_ERR_NULL;
+  if (!rows) return STS_ERR_NULL;
+  if (rows->len != shape->T) return STS_ERR_SHAPE;
+  if (!rows->top_k || !rows->top_p || !rows->min_p) return STS_ERR_NULL;
+  STS_TRY(check_ws(ws, ws_bytes, filter_bytes(shape)));
+  DeviceInfo dev;
+  STS_TRY(device_info(dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+  int32_t* flags = reinterpret_cast<int32_t*>(wsb + sizeof(WsHeader));
+  STS_TRY(reset_header(ws, st));
+  launch_validate(nullptr, nullptr, rows->top_p, rows->min_p, shape->T, shape->V, flags, hdr, false, st);
+  STS_CUDA(cudaGetLastError());
+  ResolveArgs a{};
+  a.S = S;
+  a.ld = shape->V;
+  a.rows = (int)shape->T;
+  a.V = (int)shape->V;
+  a.mode = kModeFilter;
+  a.top_k = rows->top_k;
+  a.top_p = rows->top_p;
+  a.min_p = rows->min_p;
+  a.row_flags = flags;
+  a.flags_out = nullptr;
+  a.support_size = support_size;
+  a.cut_logit = cut_logit;
+  a.cut_id = cut_id;
+  a.mask = mask;
+  a.hdr = hdr;
+  STS_CUDA(launch_resolve(a, dev.sms, st));
+  return STS_OK;
+}
+
+sts_status sts_scaled_logits(const sts_shape* shape, const void* H, const void* W,
+                             const float* temperature, int64_t t0, int64_t nrows, int64_t v0,
+                             int64_t cols, float* S_out, int64_t ld, sts_stream_t stream) {
+  if (!shape_ok(shape)) return STS_ERR_SHAPE;
+  if (!H || !W || !temperature || !S_out) return STS_ERR_NULL;
+  if (t0 < 0 || nrows < 1 || t0 + nrows > shape->T || (t0 % GEMM_BM) != 0) return STS_ERR_SHAPE;
+  if (v0 < 0 || cols < 1 || v0 + cols > shape->V || (v0 % GEMM_BN) != 0) return STS_ERR_SHAPE;
+  if (ld < cols || (ld % 4) != 0 || !aligned16(S_out) || !aligned16(H) || !aligned16(W))
+    return STS_ERR_SHAPE;
+  DeviceInfo dev;
+  STS_TRY(device_info(dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t d = shape->d;
+  CUtensorMap ma, mb, mc;
+  if (!map_kmajor(&ma, H, d, shape->T, d, GEMM_BM) || !map_kmajor(&mb, W, d, shape->V, d, GEMM_BN) ||
+      !map_out_f32(&mc, S_out, cols, nrows, ld))
+    return STS_ERR_CUDA;
+  GemmParams p{};
+  p.M = (int)nrows;
+  p.N = (int)cols;
+  p.K = (int)d;
+  p.a_mn0 = (int)t0;
+  p.b_mn0 = (int)v0;
+  p.tau = temperature + t0;
+  p.err = nullptr;  // no workspace: a bounded-wait timeout here is not reported
+  STS_CUDA((run_gemm<false, false, kEpiLogits>(ma, mb, mc, p, dev.sms, st)));
+  return STS_OK;
+}
+
+sts_status sts_get_status(const void* ws, sts_stream_t stream, int64_t* first_bad_row) {
+  if (first_bad_row) *first_bad_row = -1;
+  if (!ws) return STS_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return STS_ERR_CUDA;
+  WsHeader h;
+  if (cudaMemcpy(&h, ws, 16, cudaMemcpyDeviceToHost) != cudaSuccess) return STS_ERR_CUDA;
+  if (h.bad_row_code != ~0ull) {
+    if (first_bad_row) *first_bad_row = (int64_t)(h.bad_row_code >> 32);
+    return (sts_status)(h.bad_row_code & 0xFFFFFFFFull);
+  }
+  if (h.err) return (sts_status)h.err;
+  return STS_OK;
+}
+
+}  // extern "C"

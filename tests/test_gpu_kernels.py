@@ -1,0 +1,184 @@
+"""Kernel-level GPU tests through the C ABI: the tcgen05 logits GEMM (first
+pass of the forward) and the exact support resolver (filter hook), each
+against an independent reference on the same inputs."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from helpers import bf16_tensor, f32_values
+
+pytestmark = pytest.mark.gpu
+
+
+def _rand_hw(seed, T, d, V):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    H = workloads.f32_to_bf16_bits(rng.standard_normal((T, d), dtype=np.float32))
+    W = workloads.f32_to_bf16_bits(rng.standard_normal((V, d), dtype=np.float32)
+                                   * np.float32(1 / math.sqrt(d)))
+    tau = rng.uniform(0.5, 1.5, T).astype(np.float32)
+    return H, W, tau
+
+
+@pytest.mark.parametrize("T,d,V", [(128, 64, 256), (300, 136, 1000), (513, 1024, 4100), (64, 8, 7),
+                                   (1, 2048, 300)])
+def test_scaled_logits_against_float64(cuda_lib, T, d, V):
+    """S = (H . W^T) / tau with fp32 accumulation against the float64 product of
+    the same bf16 values (ragged M, N and K tails included)."""
+    sts = cuda_lib
+    H, W, tau = _rand_hw(10 + T + d + V, T, d, V)
+    Hd, Wd = bf16_tensor(H), bf16_tensor(W)
+    taud = torch.from_numpy(tau).cuda()
+    S = sts.sts_scaled_logits(Hd, Wd, taud).cpu().numpy()
+    ref = oracle.scaled_logits(f32_values(H), f32_values(W), tau)
+    # fp32 accumulation of d products of magnitude ~1/sqrt(d): error ~ sqrt(d) ulp
+    err = np.abs(S - ref).max()
+    assert err < 2e-5 * max(1.0, math.sqrt(d) / 8), err
+    # the division is the IEEE fp32 quotient of the fp32 accumulator: re-dividing
+    # the recovered product reproduces S exactly for the vast majority of entries
+    assert np.isfinite(S).all()
+
+
+def test_scaled_logits_sub_block_is_bit_identical(cuda_lib):
+    """A tile computed inside a sub-block launch equals the same tile of the full
+    launch bit for bit: the backward's recompute can trust the forward's cuts."""
+    sts = cuda_lib
+    T, d, V = 384, 520, 1300
+    H, W, tau = _rand_hw(3, T, d, V)
+    Hd, Wd = bf16_tensor(H), bf16_tensor(W)
+    taud = torch.from_numpy(tau).cuda()
+    full = sts.sts_scaled_logits(Hd, Wd, taud)
+    sub = sts.sts_scaled_logits(Hd, Wd, taud, t0=128, rows=200, v0=256, cols=700)
+    assert torch.equal(full[128:328, 256:956], sub)
+    sub2 = sts.sts_scaled_logits(Hd, Wd, taud, t0=256, rows=128, v0=1024, cols=276)
+    assert torch.equal(full[256:384, 1024:1300], sub2)
+
+
+def test_scaled_logits_large_k(cuda_lib):
+    """Long K loop (d = 5120, the headline hidden size) over several M/N tiles."""
+    sts = cuda_lib
+    T, d, V = 256, 5120, 768
+    H, W, tau = _rand_hw(4, T, d, V)
+    S = sts.sts_scaled_logits(bf16_tensor(H), bf16_tensor(W), torch.from_numpy(tau).cuda())
+    ref = oracle.scaled_logits(f32_values(H), f32_values(W), tau)
+    assert np.abs(S.cpu().numpy() - ref).max() < 1e-4
+
+
+# --------------------------------------------------------------------------
+# the support program on given fp32 logits: bit-exact against the oracle
+
+
+def _filter_case():
+    """Rows built to reach every branch of the resolver (V = 20000 > the
+    4096-entry candidate buffer)."""
+    rng = np.random.Generator(np.random.PCG64(77))
+    V = 20000
+    rows, meta = [], []
+
+    def add(s, k, p, mu):
+        rows.append(np.asarray(s, np.float32))
+        meta.append((k, p, mu))
+
+    for i in range(12):  # flat random rows, mixed filters
+        s = rng.standard_normal(V).astype(np.float32) / np.float32(rng.uniform(0.4, 1.6))
+        add(s, [0, 20, 50, 3000][i % 4], [1.0, 0.9, 0.5, 0.95][(i // 4) % 4], [0.0, 0.05, 0.1][i % 3])
+    for k in (1, 5, 50, 7000):  # coarse grid: many exact ties
+        s = (rng.integers(-20, 5, V) * 0.25).astype(np.float32)
+        add(s, k, 0.8, 0.0)
+    z = np.zeros(V, np.float32)  # one giant tie group: top-k and top-p inside it
+    add(z, 3, 1.0, 0.0)
+    add(z, 0, 0.5, 0.0)
+    add(z, 12345, 0.7, 0.0)
+    dense = (1.0 + np.arange(V) * 2.0 ** -20).astype(np.float32)[rng.permutation(V)]
+    add(dense, 10000, 0.5, 0.0)  # distinct values packed into very few buckets
+    add(dense, 0, 0.3, 0.0)
+    tie_max = rng.standard_normal(V).astype(np.float32)
+    tie_max[[5, 900, 19999]] = tie_max.max() + 1.0
+    add(tie_max, 1, 1.0, 0.0)
+    add(tie_max, 0, 1.0, 1.0)
+    signed0 = np.where(rng.random(V) < 0.5, np.float32(0.0), np.float32(-0.0)).astype(np.float32)
+    signed0[:100] = 1.0
+    add(signed0, 150, 1.0, 0.0)
+    tail = rng.standard_normal(V).astype(np.float32)
+    tail[V // 2:] -= 80.0  # far tail beyond the level-0 bucket range
+    add(tail, 0, 0.9999, 0.0)
+    add(tail, 15000, 1.0, 0.0)
+    add(rng.standard_normal(V).astype(np.float32) * 6, 0, 1e-6, 0.0)
+    add(rng.standard_normal(V).astype(np.float32), 0, float(np.nextafter(np.float32(1), np.float32(0))), 0.0)
+    add(rng.standard_normal(V).astype(np.float32), V, 1.0, 0.0)
+    add(rng.standard_normal(V).astype(np.float32), -3, 1.0, 0.01)
+    S = np.stack(rows)
+    T = S.shape[0]
+    md = {
+        "top_k": np.array([m[0] for m in meta], np.int32),
+        "top_p": np.array([m[1] for m in meta], np.float32),
+        "min_p": np.array([m[2] for m in meta], np.float32),
+        "temperature": np.ones(T, np.float32),
+        "target": np.zeros(T, np.int64),
+    }
+    return S, md
+
+
+def test_filter_bit_exact_against_oracle(cuda_lib):
+    sts = cuda_lib
+    S, md = _filter_case()
+    T, V = S.shape
+    out = sts.sts_filter_logits(torch.from_numpy(S).cuda(), torch.from_numpy(md["top_k"]).cuda(),
+                                torch.from_numpy(md["top_p"]).cuda(),
+                                torch.from_numpy(md["min_p"]).cuda(), want_mask=True, check=True)
+    ref = oracle.filter_rows(S, md, want_mask=True)
+    size = out["size"].cpu().numpy()
+    cid = out["cut_id"].cpu().numpy()
+    cval = out["cut_logit"].cpu().numpy()
+    mask = out["mask"].cpu().numpy().astype(bool)
+    bad = [t for t in range(T) if size[t] != ref["size"][t] or cid[t] != ref["cut_id"][t]]
+    assert not bad, [(t, size[t], ref["size"][t], cid[t], ref["cut_id"][t]) for t in bad]
+    assert np.array_equal(cval, S[np.arange(T), ref["cut_id"]])
+    assert np.array_equal(mask, ref["mask"])
+
+
+def test_filter_flat_rows_full_vocab(cuda_lib):
+    """Headline-shaped flat rows (V = 152064, s ~ N(0, 1/tau^2)): top-p keeps
+    tens of thousands of tokens; the cut must still be exact."""
+    sts = cuda_lib
+    rng = np.random.Generator(np.random.PCG64(78))
+    T, V = 24, 152064
+    S = (rng.standard_normal((T, V), dtype=np.float32)
+         / rng.uniform(0.5, 1.5, T).astype(np.float32)[:, None])
+    md = {
+        "top_k": np.where(np.arange(T) % 3 == 0, 50, 0).astype(np.int32),
+        "top_p": rng.uniform(0.8, 1.0, T).astype(np.float32),
+        "min_p": np.where(np.arange(T) % 2 == 0, 0.05, 0.0).astype(np.float32),
+        "temperature": np.ones(T, np.float32),
+        "target": np.zeros(T, np.int64),
+    }
+    md["top_p"][::5] = 1.0
+    out = sts.sts_filter_logits(torch.from_numpy(S).cuda(), torch.from_numpy(md["top_k"]).cuda(),
+                                torch.from_numpy(md["top_p"]).cuda(),
+                                torch.from_numpy(md["min_p"]).cuda(), check=True)
+    ref = oracle.filter_rows(S, md)
+    gaps = oracle.row_gaps(S, md).min(axis=1)
+    size = out["size"].cpu().numpy()
+    cid = out["cut_id"].cpu().numpy()
+    mism = (size != ref["size"]) | (cid != ref["cut_id"])
+    # a mismatch is only acceptable where float64 summation order could decide it
+    assert not (mism & (gaps > 1e-12)).any(), np.flatnonzero(mism)
+
+
+def test_filter_rejects_bad_rows(cuda_lib):
+    sts = cuda_lib
+    T, V = 4, 100
+    S = torch.randn(T, V, device="cuda")
+    k = torch.zeros(T, dtype=torch.int32, device="cuda")
+    p = torch.tensor([1.0, 0.0, 0.5, 1.5], device="cuda")
+    mu = torch.tensor([0.0, 0.0, -0.1, 0.0], device="cuda")
+    ws = torch.empty(sts.sts_workspace_bytes(T, 8, V, 2), dtype=torch.uint8, device="cuda")
+    out = sts.sts_filter_logits(S, k, p, mu, ws=ws)
+    status, row = sts.sts_get_status(ws)
+    assert (status, row) == (6, 1)  # STS_ERR_TOP_P, reported at the first bad row
+    size = out["size"].cpu().tolist()
+    assert size[0] == V and size[1] == 0 and size[2] == 0 and size[3] == 0
