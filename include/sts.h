@@ -159,6 +159,13 @@ sts_status sts_scaled_logits(const sts_shape* shape, const void* H_bf16, const v
                              const float* temperature, int64_t t0, int64_t rows, int64_t v0,
                              int64_t cols, float* S_out, int64_t ld, sts_stream_t stream);
 
+/* Test hook: the resolver's token-mass function exp(s[i] - m) (float64,
+ * table-driven) and the CUDA library exp(s[i] - m) on the same inputs, for
+ * i < n. s is a device array of fp32 logits <= m; mass and lib_exp are device
+ * arrays of n doubles. Allocates nothing. */
+sts_status sts_probe_mass_exp(const float* s, float m, double* mass, double* lib_exp, int64_t n,
+                              sts_stream_t stream);
+
 /* Synchronise the stream and read the status word a previous call left in
  * ws. first_bad_row (may be NULL) receives the lowest failing row or -1. */
 sts_status sts_get_status(const void* ws, sts_stream_t stream, int64_t* first_bad_row);

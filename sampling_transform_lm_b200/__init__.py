@@ -33,6 +33,7 @@ __all__ = [
     "sts_scaled_logits",
     "sts_get_status",
     "sts_status_string",
+    "sts_probe_mass_exp",
     "ROW_TARGET_IN_SUPPORT",
     "ROW_INVALID",
     "ROW_IDENTITY",
@@ -61,6 +62,7 @@ EXPORTED_SYMBOLS = (
     "sts_get_status",
     "sts_status_string",
     "sts_abi_version",
+    "sts_probe_mass_exp",
 )
 
 
@@ -124,6 +126,8 @@ def load():
     lib.sts_get_status.restype = ctypes.c_int
     lib.sts_status_string.argtypes = [ctypes.c_int]
     lib.sts_status_string.restype = ctypes.c_char_p
+    lib.sts_probe_mass_exp.argtypes = [P, ctypes.c_float, P, P, I64, P]
+    lib.sts_probe_mass_exp.restype = ctypes.c_int
     lib.sts_abi_version.argtypes = []
     lib.sts_abi_version.restype = ctypes.c_int
     _lib = lib
@@ -331,6 +335,18 @@ def sts_scaled_logits(H, W, temperature, t0=0, rows=None, v0=0, cols=None, *, ou
                                _stream(stream))
     _check(st, "sts_scaled_logits")
     return out[:, :cols]
+
+
+def sts_probe_mass_exp(s, m, *, stream=None):
+    """The resolver's float64 token mass exp(s - m) next to the CUDA library exp."""
+    lib = load()
+    _need(s, torch.float32, "s")
+    n = s.numel()
+    mass = torch.empty(n, dtype=torch.float64, device=s.device)
+    ref = torch.empty(n, dtype=torch.float64, device=s.device)
+    _check(lib.sts_probe_mass_exp(_ptr(s), float(m), _ptr(mass), _ptr(ref), n, _stream(stream)),
+           "sts_probe_mass_exp")
+    return mass, ref
 
 
 def sts_get_status(ws, stream=None, raise_on_error=False):

@@ -64,6 +64,8 @@ struct GemmParams {
   const int32_t* flags;
   int col_base;  // global vocabulary id of problem column 0 (kEpiDZ)
   int* err;      // STS_ERR_TIMEOUT lands here
+  float* max_part;  // kEpiLogits: per-(row, 256-column tile) max, [M][max_ld]; may be null
+  int max_ld;
 };
 
 __device__ __forceinline__ void gemm_tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
@@ -273,6 +275,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
       }
 
+      float tile_max = -INFINITY;
       for (int cc = 0; cc < GEMM_BN / CW; ++cc) {
         const int ncol0 = nb * GEMM_BN + cc * CW;  // first problem column of this chunk
         if (ncol0 >= p.N) break;
@@ -295,6 +298,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (EPI == kEpiLogits) {
 #pragma unroll
           for (int j = 0; j < CW; ++j) v[j] = __fdiv_rn(v[j], tau);
+          const int valid = p.N - ncol0;  // columns past N hold zero-filled products
+#pragma unroll
+          for (int j = 0; j < CW; ++j)
+            if (j < valid) tile_max = fmaxf(tile_max, v[j]);
         } else if (EPI == kEpiDZ) {
           if (coef != 0.f) {
             const long long col0 = (long long)p.col_base + ncol0;
@@ -345,6 +352,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         __syncwarp();
         sel ^= 1;
       }
+      if (EPI == kEpiLogits && p.max_part != nullptr && row_ok)
+        p.max_part[(size_t)row * p.max_ld + nb] = tile_max;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));

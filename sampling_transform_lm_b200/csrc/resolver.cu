@@ -4,28 +4,38 @@
 // sampling-transform scoring on one shared chunked core; implement
 // top-k/top-p/min-p replay for generic ce_modes", xorl PR 74, "What this PR
 // does", item 1) on one row of fp32 scaled logits s[0..V) held in global
-// memory (L2-resident while the CTA works on it):
+// memory:
 //
 //   order      (s desc, token id asc): every token gets a distinct 64-bit
 //              composite key K = (monotone key of s) << 32 | (2^32-1 - id),
 //              so "earlier in the order" is "larger K" and ties in s are
 //              broken by the lower id.
-//   top-k      the k-th element of the order (radix select on K, refined
-//              through histograms until the boundary bucket fits in shared
-//              memory, then sorted)
+//   top-k      the k-th element of the order
 //   top-p      the first element whose inclusive running mass reaches
 //              p * Z_k (Z_k = mass of the top-k prefix; masses are
 //              exp(s - m) in float64, m the unfiltered row max)
 //   min-p      the smallest fp32 threshold t with exp(t - m) >= min_p,
-//              found by bisection over fp32 bit patterns; all s >= t kept
-//   support    the shortest of the three prefixes; its size, mass Z_S, and
-//              last element (cut) give LSE_S = m + log Z_S
+//              found by bisection over fp32 bit patterns; every s >= t kept
+//   support    the shortest of the three prefixes; its size, mass Z_S and
+//              last element (the cut) give LSE_S = m + log Z_S
 //
-// Level-0 buckets are uniform in (m - s): bucket = floor((m - s) * 128),
-// clamped to 4095 -- monotone in s, so every bucket is a contiguous run of
-// the order. A bucket too large for the 4096-entry candidate buffer is split
-// again on its composite keys (12 bits per level) until it fits; the keys
-// are distinct, so this ends after at most six levels.
+// Work per row: one streaming pass builds a 4096-bucket histogram (count and
+// float64 mass) with buckets uniform in (m - s) -- floor((m - s) * 128),
+// clamped to 4095 -- which is monotone in s, so every bucket is a contiguous
+// run of the order. The buckets that hold a cut are then gathered in one more
+// pass (from L2), sorted by composite key and scanned, which places each cut
+// exactly. A bucket too large for the 4096-entry candidate buffer is split
+// again on its composite keys (12 bits per level) until it fits; the keys are
+// distinct, so this ends after at most six levels. The row max comes from the
+// projection's epilogue (one partial max per 256-column tile) when available.
+//
+// Masses use a table-driven float64 exponential (P. T. P. Tang, "Table-driven
+// implementation of the exponential function in IEEE floating-point
+// arithmetic", ACM TOMS 15(2), 1989): exp(x) = exp(-b/128) * exp(x + b/128)
+// with b the element's bucket, the table entries computed once per CTA with
+// the CUDA library exp, and the reduced factor (|r| <= 1/128) from its
+// degree-6 Taylor polynomial, whose truncation error (< 4e-19) is below half
+// an ulp. Elements in the clamped far-tail bucket use the library exp.
 #include <cfloat>
 #include <cmath>
 
@@ -35,15 +45,17 @@ namespace sts {
 
 namespace {
 
-constexpr int RT = 512;               // threads per resolver CTA
+constexpr int RT = 512;             // threads per resolver CTA
 constexpr int NWARP = RT / 32;
-constexpr int NB = 4096;              // histogram buckets per level
-constexpr int CAP = 4096;             // candidate buffer (composite keys)
-constexpr float BIN_SCALE = 128.f;    // level-0 buckets per logit unit
+constexpr int NB = 4096;            // histogram buckets per level
+constexpr int CAP = 4096;           // candidate buffer (composite keys)
+constexpr float BIN_SCALE = 128.f;  // level-0 buckets per logit unit
 constexpr int MAX_LEVELS = 8;
+constexpr int UNROLL = 4;           // float4 loads in flight per thread
 
 struct RSmem {
   double mass[NB];
+  double tab[NB];  // exp(-b / 128)
   unsigned long long cand[CAP];
   double cq[CAP];
   int cnt[NB];
@@ -51,10 +63,8 @@ struct RSmem {
   unsigned long long red_u[NWARP];
   long long red_l[NWARP];
   float red_f[NWARP];
-  // broadcast slots
   double bd[4];
   long long bl[4];
-  unsigned long long bu[4];
   int bi[4];
   int ncand;
 };
@@ -88,7 +98,70 @@ __device__ __forceinline__ int bin0(float s, float m) {
   return b < 0 ? 0 : b;
 }
 
-__device__ __forceinline__ double qmass(float s, double m) { return exp((double)s - m); }
+// exp((double)s - (double)m) for an element in level-0 bucket b.
+__device__ __forceinline__ double qmass_b(const double* tab, float s, double md, int b) {
+  const double x = (double)s - md;
+  if (b >= NB - 1) return exp(x);
+  const double r = x + (double)b * (1.0 / 128.0);
+  double p = 1.0 / 720.0;
+  p = fma(p, r, 1.0 / 120.0);
+  p = fma(p, r, 1.0 / 24.0);
+  p = fma(p, r, 1.0 / 6.0);
+  p = fma(p, r, 0.5);
+  p = fma(p, r, 1.0);
+  p = fma(p, r, 1.0);
+  return tab[b] * p;
+}
+
+__device__ __forceinline__ double qmass(const RSmem& sm, float s, float m) {
+  return qmass_b(sm.tab, s, (double)m, bin0(s, m));
+}
+
+// ---------------------------------------------------------------- streaming
+
+// Apply f(value, index) to every element of the row. VEC: the row start is
+// 16-byte aligned, so UNROLL float4 loads per thread are kept in flight.
+template <bool VEC, typename F>
+__device__ __forceinline__ void for_each(const float* __restrict__ x, int V, F&& f) {
+  if (VEC) {
+    const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
+    const int V4 = V >> 2;
+    for (int base = 0; base < V4; base += RT * UNROLL) {
+      float4 v[UNROLL];
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        const int i = base + u * RT + (int)threadIdx.x;
+        if (i < V4) v[u] = x4[i];
+      }
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        const int i = base + u * RT + (int)threadIdx.x;
+        if (i < V4) {
+          f(v[u].x, 4 * i);
+          f(v[u].y, 4 * i + 1);
+          f(v[u].z, 4 * i + 2);
+          f(v[u].w, 4 * i + 3);
+        }
+      }
+    }
+    for (int i = 4 * V4 + (int)threadIdx.x; i < V; i += RT) f(x[i], i);
+  } else {
+    constexpr int U = 4 * UNROLL;
+    for (int base = 0; base < V; base += RT * U) {
+      float v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * RT + (int)threadIdx.x;
+        if (i < V) v[u] = x[i];
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = base + u * RT + (int)threadIdx.x;
+        if (i < V) f(v[u], i);
+      }
+    }
+  }
+}
 
 // ---------------------------------------------------------------- block reductions
 // Fixed shuffle-down trees: results are identical on every run.
@@ -164,6 +237,10 @@ __device__ unsigned long long block_ext_u(unsigned long long v, RSmem& sm) {
   return r;
 }
 
+__device__ __forceinline__ int block_min_i(int v, RSmem& sm) {
+  return (int)(~block_ext_u<true>(~(unsigned long long)(unsigned)v, sm));
+}
+
 // Exclusive scan over threads in thread order (deterministic).
 template <typename T>
 __device__ T block_exscan(T v, T* warp_tot, T& total) {
@@ -204,11 +281,15 @@ __device__ __forceinline__ bool crit_ok(int crit, long long c, double mss, long 
   return crit == kCount ? (c >= need) : (crit == kMassGE ? (mss >= target) : (mss > target));
 }
 
+__device__ __forceinline__ void take_earlier(Cut& best, const Cut& c) {
+  if (c.K > best.K) best = c;
+}
+
 // Over the NB buckets in sm.cnt / sm.mass (bucket 0 = earliest in the order),
 // pick the first bucket where (above + inclusive prefix) meets the criterion,
 // or the last non-empty bucket if none does. Returns it with the count and
 // mass of everything before it (above included).
-__device__ void pick_bucket(RSmem& sm, int crit, long long need, double target, long long above_cnt,
+__device__ __noinline__ void pick_bucket(RSmem& sm, int crit, long long need, double target, long long above_cnt,
                             double above_mass, int& b_out, long long& cnt_excl, double& mass_excl) {
   constexpr int PER = NB / RT;
   const int base = threadIdx.x * PER;
@@ -225,7 +306,6 @@ __device__ void pick_bucket(RSmem& sm, int crit, long long need, double target, 
   double tm;
   const long long pc = block_exscan<long long>(lc, sm.red_l, tc);
   const double pm = block_exscan<double>(lm, sm.red_d, tm);
-  // first satisfying bucket owned by this thread
   int mine = NB;
   {
     long long c = above_cnt + pc;
@@ -239,7 +319,7 @@ __device__ void pick_bucket(RSmem& sm, int crit, long long need, double target, 
       }
     }
   }
-  int b = (int)(~block_ext_u<true>(~(unsigned long long)(unsigned)mine, sm));  // min
+  int b = block_min_i(mine, sm);
   if (b >= NB) b = (int)block_ext_u<true>((unsigned long long)(unsigned)(last_nz + 1), sm) - 1;
   if (b < 0) b = 0;
   if (threadIdx.x == b / PER) {
@@ -259,30 +339,115 @@ __device__ void pick_bucket(RSmem& sm, int crit, long long need, double target, 
   __syncthreads();
 }
 
-// Level-0 histogram of the row (counts and float64 masses per bucket).
-__device__ void build_hist0(RSmem& sm, const float* __restrict__ x, int V, float m) {
+// Count and mass of every bucket before bucket b (b may be NB: all buckets).
+__device__ __noinline__ void bucket_prefix(RSmem& sm, int b, long long& cnt_excl, double& mass_excl) {
+  constexpr int PER = NB / RT;
+  const int base = threadIdx.x * PER;
+  long long lc = 0;
+  double lm = 0.0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    if (base + i < b) {
+      lc += sm.cnt[base + i];
+      lm += sm.mass[base + i];
+    }
+  }
+  cnt_excl = block_sum_l(lc, sm);
+  mass_excl = block_sum_d(lm, sm);
+}
+
+// Level-0 histogram of the row (counts and float64 masses per bucket); also
+// the total mass and the last element of the order when asked.
+template <bool VEC>
+__device__ __noinline__ void build_hist0(RSmem& sm, const float* __restrict__ x, int V, float m, double* Z,
+                            unsigned long long* Kmin) {
   for (int i = threadIdx.x; i < NB; i += RT) {
     sm.cnt[i] = 0;
     sm.mass[i] = 0.0;
   }
   __syncthreads();
   const double md = (double)m;
-  for (int i = threadIdx.x; i < V; i += RT) {
-    const float s = x[i];
+  double zl = 0.0;
+  unsigned long long kl = ~0ull;
+  for_each<VEC>(x, V, [&](float s, int i) {
     const int b = bin0(s, m);
+    const double q = qmass_b(sm.tab, s, md, b);
     atomicAdd(&sm.cnt[b], 1);
-    atomicAdd(&sm.mass[b], qmass(s, md));
+    atomicAdd(&sm.mass[b], q);
+    zl += q;
+    const unsigned long long K = ckey(s, i);
+    kl = K < kl ? K : kl;
+  });
+  __syncthreads();
+  if (Z) *Z = block_sum_d(zl, sm);
+  if (Kmin) *Kmin = block_ext_u<false>(kl, sm);
+}
+
+// Sort sm.cand[0..n) descending (composite keys are distinct) and write the
+// inclusive float64 prefix of the masses to sm.cq (thread order, deterministic).
+__device__ __noinline__ void sort_and_scan(RSmem& sm, int n, float m) {
+  int n2 = 2;
+  while (n2 < n) n2 <<= 1;
+  for (int i = n + (int)threadIdx.x; i < n2; i += RT) sm.cand[i] = 0ull;  // sorts last
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += RT) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long a = sm.cand[i], c = sm.cand[ixj];
+          const bool desc = (i & k) == 0;
+          if (desc ? (a < c) : (a > c)) {
+            sm.cand[i] = c;
+            sm.cand[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
   }
+  constexpr int PER = CAP / RT;
+  const int base = threadIdx.x * PER;
+  double loc[PER];
+  double run = 0.0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int j = base + i;
+    const double qv = j < n ? qmass(sm, ckey_value(sm.cand[j]), m) : 0.0;
+    run += qv;
+    loc[i] = run;
+  }
+  double tot;
+  const double off = block_exscan<double>(run, sm.red_d, tot);
+#pragma unroll
+  for (int i = 0; i < PER; ++i) sm.cq[base + i] = off + loc[i];
   __syncthreads();
 }
 
-// Find the element of the (s desc, id asc) order where the criterion is first
-// met. Returns false (and sets *overflow) only if the refinement bound is hit.
-__device__ bool locate(RSmem& sm, const float* __restrict__ x, int V, float m, bool& hist_valid,
+// First j in [lo, hi) with C(j) = base_mass + (cq[j] - cq_before) meeting a
+// mass criterion; hi - 1 if none does.
+__device__ __noinline__ int first_mass_hit(RSmem& sm, int lo, int hi, double base_mass, double cq_before, int crit,
+                              double target) {
+  int mine = CAP;
+  for (int j = lo + (int)threadIdx.x; j < hi; j += RT) {
+    if (crit_ok(crit, 0, base_mass + (sm.cq[j] - cq_before), 0, target)) {
+      mine = j;
+      break;
+    }
+  }
+  int j = block_min_i(mine, sm);
+  if (j >= hi) j = hi - 1;
+  return j;
+}
+
+// General search: the element of the order where the criterion is first met,
+// refining oversized buckets. Returns false if the refinement bound is hit.
+template <bool VEC>
+__device__ __noinline__ bool locate(RSmem& sm, const float* __restrict__ x, int V, float m, bool& hist_valid,
                        int crit, long long need, double target, Cut& out) {
   const double md = (double)m;
   if (!hist_valid) {
-    build_hist0(sm, x, V, m);
+    build_hist0<VEC>(sm, x, V, m, nullptr, nullptr);
     hist_valid = true;
   }
   int b;
@@ -296,16 +461,14 @@ __device__ bool locate(RSmem& sm, const float* __restrict__ x, int V, float m, b
 
   for (int level = 0; set_cnt > CAP; ++level) {
     if (level >= MAX_LEVELS) return false;
-    // exact key range of the current set
     unsigned long long kmin = ~0ull, kmax = 0ull;
-    for (int i = threadIdx.x; i < V; i += RT) {
-      const float s = x[i];
-      if (bin0(s, m) != b) continue;
+    for_each<VEC>(x, V, [&](float s, int i) {
+      if (bin0(s, m) != b) return;
       const unsigned long long K = ckey(s, i);
-      if (refined && (K < Klo || K > Khi)) continue;
+      if (refined && (K < Klo || K > Khi)) return;
       kmin = K < kmin ? K : kmin;
       kmax = K > kmax ? K : kmax;
-    }
+    });
     Klo = block_ext_u<false>(kmin, sm);
     Khi = block_ext_u<true>(kmax, sm);
     refined = true;
@@ -318,15 +481,15 @@ __device__ bool locate(RSmem& sm, const float* __restrict__ x, int V, float m, b
     }
     hist_valid = false;
     __syncthreads();
-    for (int i = threadIdx.x; i < V; i += RT) {
-      const float s = x[i];
-      if (bin0(s, m) != b) continue;
+    for_each<VEC>(x, V, [&](float s, int i) {
+      const int b0 = bin0(s, m);
+      if (b0 != b) return;
       const unsigned long long K = ckey(s, i);
-      if (K < Klo || K > Khi) continue;
+      if (K < Klo || K > Khi) return;
       const int sb = (int)((Khi - K) >> shift);
       atomicAdd(&sm.cnt[sb], 1);
-      atomicAdd(&sm.mass[sb], qmass(s, md));
-    }
+      atomicAdd(&sm.mass[sb], qmass_b(sm.tab, s, md, b0));
+    });
     __syncthreads();
     int c;
     long long ce;
@@ -344,75 +507,24 @@ __device__ bool locate(RSmem& sm, const float* __restrict__ x, int V, float m, b
     __syncthreads();
   }
 
-  // gather the boundary set
   if (threadIdx.x == 0) sm.ncand = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < V; i += RT) {
-    const float s = x[i];
-    if (bin0(s, m) != b) continue;
+  for_each<VEC>(x, V, [&](float s, int i) {
+    if (bin0(s, m) != b) return;
     const unsigned long long K = ckey(s, i);
-    if (refined && (K < Klo || K > Khi)) continue;
+    if (refined && (K < Klo || K > Khi)) return;
     const int slot = atomicAdd(&sm.ncand, 1);
     if (slot < CAP) sm.cand[slot] = K;
-  }
+  });
   __syncthreads();
   const int n = min(sm.ncand, CAP);
-  int n2 = 2;
-  while (n2 < n) n2 <<= 1;
-  for (int i = n + (int)threadIdx.x; i < n2; i += RT) sm.cand[i] = 0ull;  // sorts last
-  __syncthreads();
-  // bitonic sort, descending
-  for (int k = 2; k <= n2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += RT) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long a = sm.cand[i], c = sm.cand[ixj];
-          const bool desc = (i & k) == 0;
-          if (desc ? (a < c) : (a > c)) {
-            sm.cand[i] = c;
-            sm.cand[ixj] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  // inclusive scan of masses in sorted order (8 per thread, thread order)
-  constexpr int PER = CAP / RT;
-  const int base = threadIdx.x * PER;
-  double loc[PER];
-  double run = 0.0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int j = base + i;
-    const double qv = j < n ? qmass(ckey_value(sm.cand[j]), md) : 0.0;
-    run += qv;
-    loc[i] = run;
-  }
-  double tot;
-  const double off = block_exscan<double>(run, sm.red_d, tot);
-#pragma unroll
-  for (int i = 0; i < PER; ++i) sm.cq[base + i] = off + loc[i];
-  __syncthreads();
-
+  sort_and_scan(sm, n, m);
   int jstar;
-  if (crit == kCount) {
+  if (crit == kCount)
     jstar = (int)(need - above_cnt - 1);
-  } else {
-    int mine = CAP;
-    for (int i = 0; i < PER; ++i) {
-      const int j = base + i;
-      if (j < n && crit_ok(crit, 0, above_mass + sm.cq[j], 0, target)) {
-        mine = j;
-        break;
-      }
-    }
-    jstar = (int)(~block_ext_u<true>(~(unsigned long long)(unsigned)mine, sm));
-    if (jstar >= n) jstar = n - 1;
-  }
-  if (jstar < 0) jstar = 0;
-  if (jstar > n - 1) jstar = n - 1;
+  else
+    jstar = first_mass_hit(sm, 0, n, above_mass, 0.0, crit, target);
+  jstar = max(0, min(jstar, n - 1));
   out.K = sm.cand[jstar];
   out.cnt = above_cnt + jstar + 1;
   out.mass = above_mass + sm.cq[jstar];
@@ -420,12 +532,29 @@ __device__ bool locate(RSmem& sm, const float* __restrict__ x, int V, float m, b
   return true;
 }
 
-__device__ __forceinline__ void take_earlier(Cut& best, const Cut& c) {
-  if (c.K > best.K) best = c;
+// The prefix kept by min-p: every element with key >= kt (one pass).
+template <bool VEC>
+__device__ __noinline__ Cut min_p_cut_pass(RSmem& sm, const float* __restrict__ x, int V, float m, uint32_t kt) {
+  long long c = 0;
+  double ms = 0.0;
+  unsigned long long kl = ~0ull;
+  for_each<VEC>(x, V, [&](float s, int i) {
+    if (key32(s) >= kt) {
+      ++c;
+      ms += qmass(sm, s, m);
+      const unsigned long long K = ckey(s, i);
+      kl = K < kl ? K : kl;
+    }
+  });
+  Cut cm;
+  cm.K = block_ext_u<false>(kl, sm);
+  cm.cnt = block_sum_l(c, sm);
+  cm.mass = block_sum_d(ms, sm);
+  return cm;
 }
 
 // Smallest fp32 t (as a key) with exp(t - m) >= mu, mu in (0, 1].
-__device__ uint32_t min_p_threshold_key(float m, float mu) {
+__device__ __noinline__ uint32_t min_p_threshold_key(float m, float mu) {
   uint32_t lo = key32(-FLT_MAX), hi = key32(m);  // P(lo) false, P(hi) true
   const double md = (double)m, mud = (double)mu;
   if (exp((double)(-FLT_MAX) - md) >= mud) return lo;
@@ -439,10 +568,63 @@ __device__ uint32_t min_p_threshold_key(float m, float mu) {
   return hi;
 }
 
-__global__ void __launch_bounds__(RT) resolve_kernel(const ResolveArgs a) {
+template <bool VEC>
+__device__ __noinline__ float row_max_pass(const float* __restrict__ x, int V) {
+  float lm = -INFINITY;
+  for_each<VEC>(x, V, [&](float s, int) { lm = fmaxf(lm, s); });
+  return lm;
+}
+
+// Gather every element of buckets [0, bk] into sm.cand; returns the count.
+template <bool VEC>
+__device__ __noinline__ int gather_prefix(RSmem& sm, const float* __restrict__ x, int V, float m,
+                                          int bk) {
+  if (threadIdx.x == 0) sm.ncand = 0;
+  __syncthreads();
+  for_each<VEC>(x, V, [&](float s, int i) {
+    if (bin0(s, m) > bk) return;
+    const int slot = atomicAdd(&sm.ncand, 1);
+    if (slot < CAP) sm.cand[slot] = ckey(s, i);
+  });
+  __syncthreads();
+  const int n = min(sm.ncand, CAP);
+  __syncthreads();
+  return n;
+}
+
+// Gather the elements of buckets bp and bm (either may be -1) into sm.cand
+// and, when kt is live, return the last element with key >= kt among the
+// buckets up to bm (the end of the min-p prefix).
+template <bool VEC>
+__device__ __noinline__ int gather_two(RSmem& sm, const float* __restrict__ x, int V, float m,
+                                       int bp, int bm, bool mu_on, uint32_t kt,
+                                       unsigned long long* K_mu) {
+  if (threadIdx.x == 0) sm.ncand = 0;
+  __syncthreads();
+  unsigned long long kl = ~0ull;
+  for_each<VEC>(x, V, [&](float s, int i) {
+    const int b0 = bin0(s, m);
+    if (mu_on && b0 <= bm && key32(s) >= kt) {
+      const unsigned long long K = ckey(s, i);
+      kl = K < kl ? K : kl;
+    }
+    if (b0 != bp && b0 != bm) return;
+    const int slot = atomicAdd(&sm.ncand, 1);
+    if (slot < CAP) sm.cand[slot] = ckey(s, i);
+  });
+  *K_mu = block_ext_u<false>(kl, sm);
+  const int n = min(sm.ncand, CAP);
+  __syncthreads();
+  return n;
+}
+
+template <bool VEC>
+__global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   RSmem& sm = *reinterpret_cast<RSmem*>(smem_raw);
   const int V = a.V;
+  for (int i = threadIdx.x; i < NB; i += RT) sm.tab[i] = exp(-(double)i * (1.0 / 128.0));
+  __syncthreads();
 
   for (int r = blockIdx.x; r < a.rows; r += gridDim.x) {
     const float* __restrict__ x = a.S + (size_t)r * (size_t)a.ld;
@@ -461,28 +643,26 @@ __global__ void __launch_bounds__(RT) resolve_kernel(const ResolveArgs a) {
       }
       if (a.mask)
         for (int i = threadIdx.x; i < V; i += RT) a.mask[(size_t)r * V + i] = 0;
+      __syncthreads();
       continue;
     }
 
-    // unfiltered row max
+    // unfiltered row max: from the projection's per-tile maxima when present
     float lm = -INFINITY;
-    for (int i = threadIdx.x; i < V; i += RT) lm = fmaxf(lm, x[i]);
+    if (a.max_part) {
+      const float* mp = a.max_part + (size_t)r * (size_t)a.n_parts;
+      for (int i = threadIdx.x; i < a.n_parts; i += RT) lm = fmaxf(lm, mp[i]);
+    } else {
+      lm = row_max_pass<VEC>(x, V);
+    }
     const float m = block_max_f(lm, sm);
     const double md = (double)m;
 
-    // level-0 histogram, total mass and the last element of the order
-    build_hist0(sm, x, V, m);
+    double Z;
+    unsigned long long Klast;
+    build_hist0<VEC>(sm, x, V, m, &Z, &Klast);
     bool hist_valid = true;
-    double zl = 0.0;
-    unsigned long long kmin = ~0ull;
-    for (int i = threadIdx.x; i < V; i += RT) {
-      const float s = x[i];
-      zl += qmass(s, md);
-      const unsigned long long K = ckey(s, i);
-      kmin = K < kmin ? K : kmin;
-    }
-    const double Z = block_sum_d(zl, sm);
-    Cut best{block_ext_u<false>(kmin, sm), (long long)V, Z};
+    Cut best{Klast, (long long)V, Z};
 
     const int k = a.top_k[r];
     const float p = a.top_p[r];
@@ -492,38 +672,102 @@ __global__ void __launch_bounds__(RT) resolve_kernel(const ResolveArgs a) {
     const bool mu_on = mu > 0.0f;
     bool ok = true;
 
-    double Zk = Z;
-    if (k_on) {
-      Cut ck;
-      ok = ok && locate(sm, x, V, m, hist_valid, kCount, (long long)k, 0.0, ck);
-      Zk = ck.mass;
-      take_earlier(best, ck);
-    }
-    if (ok && p_on) {
-      Cut cp;
-      ok = ok && locate(sm, x, V, m, hist_valid, kMassGE, 0, (double)p * Zk, cp);
-      take_earlier(best, cp);
-    }
-    if (ok && mu_on) {
+    uint32_t kt = 0;
+    if (mu_on) {
       if (threadIdx.x == 0) sm.bi[0] = (int)min_p_threshold_key(m, mu);
       __syncthreads();
-      const uint32_t kt = (uint32_t)sm.bi[0];
+      kt = (uint32_t)sm.bi[0];
       __syncthreads();
-      long long c = 0;
-      double ms = 0.0;
-      unsigned long long kl = ~0ull;
-      for (int i = threadIdx.x; i < V; i += RT) {
-        const float s = x[i];
-        if (key32(s) >= kt) {
-          ++c;
-          ms += qmass(s, md);
-          const unsigned long long K = ckey(s, i);
-          kl = K < kl ? K : kl;
+    }
+
+    bool done = false;
+    double Zk = Z;
+    if (k_on) {
+      int bk;
+      long long ce;
+      double me;
+      pick_bucket(sm, kCount, (long long)k, 0.0, 0, 0.0, bk, ce, me);
+      const long long incl = ce + sm.cnt[bk];
+      __syncthreads();
+      if (incl <= CAP) {
+        // small k: the whole prefix of buckets [0, bk] fits, and every cut
+        // that can be earlier than the top-k cut lies inside it
+        const int n = gather_prefix<VEC>(sm, x, V, m, bk);
+        sort_and_scan(sm, n, m);
+        const int jk = min(k, n) - 1;
+        Cut ck{sm.cand[jk], (long long)jk + 1, sm.cq[jk]};
+        Zk = ck.mass;
+        take_earlier(best, ck);
+        if (p_on) {
+          const int jp = first_mass_hit(sm, 0, jk + 1, 0.0, 0.0, kMassGE, (double)p * Zk);
+          take_earlier(best, Cut{sm.cand[jp], (long long)jp + 1, sm.cq[jp]});
         }
+        if (mu_on) {
+          // kept candidates form a prefix; count them
+          int mine = 0;
+          for (int j = threadIdx.x; j < n; j += RT) mine += (uint32_t)(sm.cand[j] >> 32) >= kt ? 1 : 0;
+          const int nk = (int)block_sum_l(mine, sm);
+          if (nk >= 1 && nk < n) take_earlier(best, Cut{sm.cand[nk - 1], (long long)nk, sm.cq[nk - 1]});
+        }
+        __syncthreads();
+        done = true;
+      } else {
+        Cut ck;
+        ok = locate<VEC>(sm, x, V, m, hist_valid, kCount, (long long)k, 0.0, ck);
+        Zk = ck.mass;
+        take_earlier(best, ck);
       }
-      Cut cm{block_ext_u<false>(kl, sm), block_sum_l(c, sm), 0.0};
-      cm.mass = block_sum_d(ms, sm);
-      take_earlier(best, cm);
+    }
+
+    if (ok && !done && (p_on || mu_on)) {
+      if (!hist_valid) {
+        build_hist0<VEC>(sm, x, V, m, nullptr, nullptr);
+        hist_valid = true;
+      }
+      const double target = (double)p * Zk;
+      int bp = -1, bm = -1;
+      long long cp_excl = 0, cm_excl = 0;
+      double mp_excl = 0.0, mm_excl = 0.0;
+      if (p_on) pick_bucket(sm, kMassGE, 0, target, 0, 0.0, bp, cp_excl, mp_excl);
+      if (mu_on) {
+        bm = bin0(key32_value(kt), m);
+        bucket_prefix(sm, bm, cm_excl, mm_excl);
+      }
+      const int np_ = bp >= 0 ? sm.cnt[bp] : 0;
+      const int nm_ = (bm >= 0 && bm != bp) ? sm.cnt[bm] : 0;
+      __syncthreads();
+      if (np_ + nm_ <= CAP) {
+        // one pass gathers both boundary buckets and the last min-p element
+        unsigned long long K_mu = 0ull;
+        const int n = gather_two<VEC>(sm, x, V, m, bp, bm, mu_on, kt, &K_mu);
+        sort_and_scan(sm, n, m);
+        // sorted candidates: the earlier bucket's run first
+        if (p_on) {
+          const int lo = (bm >= 0 && bm < bp) ? nm_ : 0;
+          const double before = lo > 0 ? sm.cq[lo - 1] : 0.0;
+          const int jp = first_mass_hit(sm, lo, lo + np_, mp_excl, before, kMassGE, target);
+          take_earlier(best, Cut{sm.cand[jp], cp_excl + (jp - lo) + 1, mp_excl + (sm.cq[jp] - before)});
+        }
+        if (mu_on) {
+          const int lo = (bp >= 0 && bp < bm) ? np_ : 0;
+          const int cntb = sm.cnt[bm];
+          int mine = 0;
+          for (int j = lo + (int)threadIdx.x; j < lo + cntb; j += RT)
+            mine += (uint32_t)(sm.cand[j] >> 32) >= kt ? 1 : 0;
+          const int nk = (int)block_sum_l(mine, sm);
+          const double before = lo > 0 ? sm.cq[lo - 1] : 0.0;
+          const double mass = mm_excl + (nk > 0 ? sm.cq[lo + nk - 1] - before : 0.0);
+          take_earlier(best, Cut{K_mu, cm_excl + nk, mass});
+        }
+        __syncthreads();
+      } else {
+        if (p_on) {
+          Cut cp;
+          ok = locate<VEC>(sm, x, V, m, hist_valid, kMassGE, 0, target, cp);
+          take_earlier(best, cp);
+        }
+        if (ok && mu_on) take_earlier(best, min_p_cut_pass<VEC>(sm, x, V, m, kt));
+      }
     }
 
     if (!ok) {
@@ -535,24 +779,22 @@ __global__ void __launch_bounds__(RT) resolve_kernel(const ResolveArgs a) {
         if (a.support_size) a.support_size[r] = 0;
         if (a.flags_out) a.flags_out[r] = STS_ROW_INVALID;
       }
+      __syncthreads();
       continue;
     }
 
     const double lse = md + log(best.mass);
-    const float cut_v = ckey_value(best.K);
-    const int cut_i = ckey_id(best.K);
-
     if (a.mode == kModeSample) {
       Cut cs;
       const double tgt = a.u[r] * best.mass;
-      const bool ok2 = locate(sm, x, V, m, hist_valid, kMassGT, 0, tgt, cs);
+      const bool ok2 = locate<VEC>(sm, x, V, m, hist_valid, kMassGT, 0, tgt, cs);
       if (!ok2 || cs.K < best.K) cs = best;
       if (threadIdx.x == 0) a.sampled[r] = ckey_id(cs.K);
     }
     if (threadIdx.x == 0) {
       if (a.support_size) a.support_size[r] = (int32_t)best.cnt;
-      if (a.cut_logit) a.cut_logit[r] = cut_v;
-      if (a.cut_id) a.cut_id[r] = cut_i;
+      if (a.cut_logit) a.cut_logit[r] = ckey_value(best.K);
+      if (a.cut_id) a.cut_id[r] = ckey_id(best.K);
       if (a.row_max) a.row_max[r] = m;
       if (a.lse_support) a.lse_support[r] = (float)lse;
       int fl = (!k_on && !p_on && !mu_on) ? STS_ROW_IDENTITY : 0;
@@ -600,6 +842,20 @@ __global__ void validate_kernel(const int64_t* target, const float* temperature,
     atomicMin(&hdr->bad_row_code, ((unsigned long long)r << 32) | (unsigned long long)code);
 }
 
+// Evaluates the resolver's mass function exp(s - m) and the library exp on
+// the same inputs (test hook for the table-driven exponential).
+__global__ void mass_probe_kernel(const float* s, float m, double* mine, double* lib, int64_t n) {
+  __shared__ double tab[NB];
+  for (int i = threadIdx.x; i < NB; i += blockDim.x) tab[i] = exp(-(double)i * (1.0 / 128.0));
+  __syncthreads();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = s[i];
+    mine[i] = qmass_b(tab, v, (double)m, bin0(v, m));
+    lib[i] = exp((double)v - (double)m);
+  }
+}
+
 }  // namespace
 
 void launch_validate(const int64_t* target, const float* temperature, const float* top_p,
@@ -613,14 +869,23 @@ void launch_validate(const int64_t* target, const float* temperature, const floa
 
 size_t resolve_smem_bytes() { return sizeof(RSmem); }
 
+cudaError_t launch_mass_probe(const float* s, float m, double* mine, double* lib, int64_t n,
+                              cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int blocks = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+  mass_probe_kernel<<<blocks, 256, 0, stream>>>(s, m, mine, lib, n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_resolve(const ResolveArgs& a, int num_sms, cudaStream_t stream) {
   const size_t smem = sizeof(RSmem);
-  cudaError_t e = cudaFuncSetAttribute(resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const bool vec = (a.ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.S) & 15u) == 0);
+  auto kern = vec ? resolve_kernel<true> : resolve_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = a.rows < num_sms ? a.rows : num_sms;
   if (grid <= 0) return cudaSuccess;
-  resolve_kernel<<<grid, RT, smem, stream>>>(a);
+  kern<<<grid, RT, smem, stream>>>(a);
   return cudaGetLastError();
 }
 

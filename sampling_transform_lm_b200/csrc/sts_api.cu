@@ -149,14 +149,17 @@ int64_t vocab_chunk(const sts_shape* s) {
   return vc < Vpad ? vc : Vpad;
 }
 
+int64_t n_parts(const sts_shape* s) { return (s->V + GEMM_BN - 1) / GEMM_BN; }
+
 struct FwdLayout {
-  size_t flags_off, logits_off, total;
+  size_t flags_off, max_off, logits_off, total;
 };
 
 FwdLayout fwd_layout(const sts_shape* s) {
   FwdLayout L;
   L.flags_off = sizeof(WsHeader);
-  L.logits_off = align_up(L.flags_off + (size_t)s->T * 4, kAlign);
+  L.max_off = align_up(L.flags_off + (size_t)s->T * 4, kAlign);
+  L.logits_off = align_up(L.max_off + (size_t)row_chunk(s) * (size_t)n_parts(s) * 4, kAlign);
   L.total = align_up(L.logits_off + (size_t)row_chunk(s) * (size_t)logits_ld(s) * 4, kAlign);
   return L;
 }
@@ -235,6 +238,8 @@ sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, co
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
   int32_t* flags = fwd ? saved->flags : reinterpret_cast<int32_t*>(wsb + L.flags_off);
   float* S = reinterpret_cast<float*>(wsb + L.logits_off);
+  float* max_part = reinterpret_cast<float*>(wsb + L.max_off);
+  const int np = (int)n_parts(shape);
 
   STS_TRY(reset_header(ws, st));
   launch_validate(rows->target, rows->temperature, rows->top_p, rows->min_p, T, V, flags, hdr, fwd, st);
@@ -255,6 +260,8 @@ sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, co
     p.a_mn0 = (int)t0;
     p.tau = rows->temperature + t0;
     p.err = &hdr->err;
+    p.max_part = max_part;
+    p.max_ld = np;
     STS_CUDA((run_gemm<false, false, kEpiLogits>(ma, mb, mc, p, dev.sms, st)));
 
     ResolveArgs a{};
@@ -282,6 +289,8 @@ sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, co
     }
     a.hdr = hdr;
     a.row_base = t0;
+    a.max_part = max_part;
+    a.n_parts = np;
     STS_CUDA(launch_resolve(a, dev.sms, st));
   }
   return STS_OK;
@@ -483,6 +492,16 @@ sts_status sts_scaled_logits(const sts_shape* shape, const void* H, const void* 
   p.tau = temperature + t0;
   p.err = nullptr;  // no workspace: a bounded-wait timeout here is not reported
   STS_CUDA((run_gemm<false, false, kEpiLogits>(ma, mb, mc, p, dev.sms, st)));
+  return STS_OK;
+}
+
+sts_status sts_probe_mass_exp(const float* s, float m, double* mass, double* lib_exp, int64_t n,
+                              sts_stream_t stream) {
+  if (!s || !mass || !lib_exp) return STS_ERR_NULL;
+  if (n < 0) return STS_ERR_SHAPE;
+  DeviceInfo dev;
+  STS_TRY(device_info(dev));
+  STS_CUDA(launch_mass_probe(s, m, mass, lib_exp, n, reinterpret_cast<cudaStream_t>(stream)));
   return STS_OK;
 }
 

@@ -52,6 +52,8 @@ struct ResolveArgs {
   uint8_t* mask;           // [rows][V]
   WsHeader* hdr;
   int64_t row_base;        // global index of the chunk's first row (error reports)
+  const float* max_part;   // [rows][n_parts] per-tile row maxima, or null (max pass)
+  int n_parts;
 };
 
 // kernels / launchers (resolver.cu)
@@ -60,5 +62,7 @@ void launch_validate(const int64_t* target, const float* temperature, const floa
                      bool check_target, cudaStream_t stream);
 cudaError_t launch_resolve(const ResolveArgs& a, int num_sms, cudaStream_t stream);
 size_t resolve_smem_bytes();
+cudaError_t launch_mass_probe(const float* s, float m, double* mine, double* lib, int64_t n,
+                              cudaStream_t stream);
 
 }  // namespace sts

@@ -44,6 +44,8 @@ def _check_forward(sts_out, s, rows, ref):
     """Forward contract; returns the rows whose gradients are comparable."""
     flagged = near_gap_rows(s, rows)
     bad, flagged_mism, max_err = compare_logprob(sts_out["logprob"], ref["logprob"], flagged)
+    print(f"{int(flagged.sum())} near-gap rows, {flagged_mism} of them differ; "
+          f"max |dlogprob| elsewhere {max_err:.2e}")
     assert sts_out["status"] == 0
     assert bad == 0, (bad, flagged_mism, max_err)
     size = sts_out["saved"]["support_size"]
@@ -99,7 +101,7 @@ def test_chunking_does_not_change_results(cuda_lib):
     for key in ("support_size", "cut_id", "cut_logit", "lse_support", "flags"):
         assert np.array_equal(a["saved"][key], b["saved"][key]), key
     assert np.array_equal(a["dW"], b["dW"])
-    assert rel_fro(b["dH"], a["dH"]) < 1e-6
+    assert rel_fro(b["dH"], a["dH"]) < 1e-5  # fp32 reduce-add across chunks vs one K loop
 
 
 def test_identity_rows_match_plain_softmax(cuda_lib):
