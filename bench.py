@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Benchmark of the sampling-transform scoring core on B200: scored tokens/s
+of one forward + backward step (per row: fp32 logits through the LM head,
+per-row temperature, top-k / top-p / min-p support, selected-token logprob,
+closed-form recompute VJP into dH and dW).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ours|reference]
+
+One process per GPU (launched with torch.distributed.run for N > 1). Every
+rank scores its own batch of T rows against the same W (weak scaling); the
+step is timed with CUDA events between barriers and the max over ranks is
+reported. Rank 0 prints one JSON line.
+
+``--impl reference`` times the float64 CPU oracle instead (rank 0 only), on
+a bounded sample of rows of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "scored tokens/s fwd+bwd at 1 B200; % of bf16 tensor-core roofline"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = 4  # T=16384, d=5120, V=152064: the headline roofline workload
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"bf16_burst": float(pk["bf16_tflops"]),
+                "bf16_sustained": float(pk["bf16_tflops_sustained"]),
+                "hbm_gbs": float(pk["hbm_gbs"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"bf16_burst": 1590.0, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0,
+                "source": "fallback"}
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (host logic, also exercised by CPU gloo tests)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        return parse_clock_lines(out)
+
+
+def parse_clock_lines(text):
+    """Median SM clock, max clock and the throttle reasons seen in the
+    nvidia-smi samples (csv, noheader, nounits; fields as ClockSampler.FIELDS)."""
+    sm, mx, reasons = [], [], set()
+    for line in text.strip().splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 7:
+            continue
+        try:
+            sm.append(float(parts[0]))
+            mx.append(float(parts[1]))
+        except ValueError:
+            continue
+        for name, val in zip(ClockSampler.REASONS, parts[3:7]):
+            if val.lower() == "active":
+                reasons.add(name)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+def clocks_rejected(clk) -> bool:
+    if clk is None:
+        return False
+    bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+    if bad & set(clk["reasons"]):
+        return True
+    return clk["sm_mhz"] < 0.5 * clk["sm_max_mhz"] and not clk["reasons"]
+
+
+def _gpu_id(torch, dev_index):
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev_index).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:  # noqa: BLE001
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[dev_index]
+        return str(dev_index)
+
+
+# --------------------------------------------------------------------------
+# the float64 oracle on the host cores (baseline / reference arm)
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [int(i.get("num_threads", 1)) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def oracle_step(data, rows_idx, Wf):
+    """One oracle forward + backward over the sampled rows (full V and d)."""
+    import oracle
+
+    Hf = workloads.bf16_to_f32(data["H"][rows_idx])
+    meta = {k: data[k][rows_idx] for k in ("temperature", "top_k", "top_p", "min_p")}
+    s = oracle.scaled_logits(Hf, Wf, meta["temperature"], vocab_slice=16384)
+    y = oracle.sample_rows(s, dict(meta, target=np.zeros(len(rows_idx), np.int64)),
+                           data["u"][rows_idx])
+    rows = dict(meta, target=y)
+    oracle.forward(None, None, rows, s=s)
+    oracle.backward(Hf, Wf, rows, np.ones(len(rows_idx)), s=s, vocab_slice=16384)
+
+
+def time_oracle(data, n_rows, steps, warmup):
+    rng = np.random.Generator(np.random.PCG64(4242))
+    T = data["workload"].T
+    Wf = workloads.bf16_to_f32(data["W"])
+    times = []
+    for i in range(warmup + steps):
+        idx = np.sort(rng.choice(T, n_rows, replace=False))
+        t0 = time.perf_counter()
+        oracle_step(data, idx, Wf)
+        if i >= warmup:
+            times.append(time.perf_counter() - t0)
+    return times
+
+
+# --------------------------------------------------------------------------
+# the CUDA path
+
+
+def run_ours(args, rank, local_rank, world):
+    import torch
+
+    import sampling_transform_lm_b200 as sts
+
+    sts.load()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks = _peaks()
+    wl = workloads.WORKLOADS[args.workload]
+    data = workloads.make(args.workload, batch=rank, T=args.rows, V=args.vocab)
+    T, d, V = data["H"].shape[0], wl.d, data["W"].shape[0]
+
+    def up(a, dt):
+        return torch.from_numpy(np.ascontiguousarray(a, dt)).to(dev)
+
+    H = up(data["H"].view(np.int16), np.int16).view(torch.bfloat16)
+    W = up(data["W"].view(np.int16), np.int16).view(torch.bfloat16)
+    tau, k, p, mu = (up(data["temperature"], np.float32), up(data["top_k"], np.int32),
+                     up(data["top_p"], np.float32), up(data["min_p"], np.float32))
+    g = up(data["g"], np.float32)
+    # replayed tokens: drawn on the GPU from each row's filtered distribution
+    y = sts.sts_sample(H, W, tau, k, p, mu, up(data["u"], np.float64), check=True)
+    ws_f = torch.empty(sts.sts_workspace_bytes(T, d, V, 0), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(sts.sts_workspace_bytes(T, d, V, 1, wl.vocab_chunk), dtype=torch.uint8,
+                       device=dev)
+    dW = torch.empty((V, d), dtype=torch.float32, device=dev)
+    dH = torch.empty((T, d), dtype=torch.float32, device=dev)
+
+    def step(Hx=H, yx=y, taux=tau, kx=k, px=p, mux=mu, gx=g):
+        lp, saved, _ = sts.sts_forward(Hx, W, yx, taux, kx, px, mux, ws=ws_f)
+        if wl.backward:
+            sts.sts_backward(Hx, W, yx, taux, kx, px, mux, saved, gx, dW=dW, dH=dH,
+                             vocab_chunk=wl.vocab_chunk, ws=ws_b)
+        return lp
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, bad = sts.sts_get_status(ws_f)
+    if st != 0:
+        raise RuntimeError(f"forward status {st} at row {bad}")
+
+    stream = torch.cuda.current_stream()
+
+    def timed_region():
+        clk = ClockSampler(_gpu_id(torch, local_rank))
+        barrier()
+        torch.cuda.synchronize()
+        clk.start()
+        time.sleep(0.3)  # let the sampler attach before load starts
+        n0 = sts.sts_launch_count()
+        sts.sts_timing_enable(True)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = e0.elapsed_time(e1) / args.steps
+        kern = sts.sts_timing_read()
+        sts.sts_timing_enable(False)
+        launches = sts.sts_launch_count() - n0
+        return ms, kern, launches, clk.stop()
+
+    ms, kern, launches, clk = timed_region()
+    if clocks_rejected(clk):
+        ms, kern, launches, clk = timed_region()  # one re-measurement
+    ms_max = reduce_max(ms, dev)
+    value = world * T / (ms_max / 1e3)
+
+    # dominant kernel and its roofline (algorithmic work over live CUDA-event time)
+    gemm_flops = 2.0 * T * d * V  # per step, per GEMM kind (summed over its chunks)
+    work = {"logits_gemm": gemm_flops, "dz_gemm": gemm_flops, "dw_gemm": gemm_flops,
+            "dh_gemm": gemm_flops}
+    dom = max(kern, key=lambda n: kern[n][0])
+    dom_ms, dom_n = kern[dom]
+    if dom in work:
+        achieved = work[dom] * args.steps / (dom_ms / 1e3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_sustained"], 4), "traffic": None,
+                "launches": dom_n, "ms_per_step": round(dom_ms / args.steps, 3),
+                "peak_note": f"bf16 sustained ({peaks['source']}); kernel timed inside a long step"}
+    else:
+        bytes_ = 4.0 * T * V  # one read of the row chunk's fp32 logits
+        achieved = bytes_ * args.steps / (dom_ms / 1e3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": None, "launches": dom_n, "ms_per_step": round(dom_ms / args.steps, 3)}
+    per_kernel = {n: round(v[0] / args.steps, 3) for n, v in kern.items() if v[1]}
+
+    # end to end through the public API: inputs from pinned host memory, the
+    # step's logprobs read back every step (W stays resident: a model weight)
+    host = {
+        "H": torch.from_numpy(data["H"].view(np.int16)).pin_memory(),
+        "y": y.cpu().pin_memory(),
+        "tau": torch.from_numpy(data["temperature"]).pin_memory(),
+        "k": torch.from_numpy(data["top_k"]).pin_memory(),
+        "p": torch.from_numpy(data["top_p"]).pin_memory(),
+        "mu": torch.from_numpy(data["min_p"]).pin_memory(),
+        "g": torch.from_numpy(data["g"]).pin_memory(),
+    }
+    dbuf = {n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in host.items()}
+    lp_host = torch.empty(T, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = lp_host.numel() * lp_host.element_size()
+
+    def e2e_step():
+        for n, t in host.items():
+            dbuf[n].copy_(t, non_blocking=True)
+        lp = step(dbuf["H"].view(torch.bfloat16), dbuf["y"], dbuf["tau"], dbuf["k"], dbuf["p"],
+                  dbuf["mu"], dbuf["g"])
+        lp_host.copy_(lp, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, dev)
+    launches_all = int(reduce_sum(launches, dev))
+
+    out = None
+    if rank == 0:
+        credited = (10.0 if wl.backward else 4.0) * T * d * V
+        executed = (8.0 if wl.backward else 2.0) * T * d * V
+        out = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_max, 3),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": f"{wl.name}: {wl.desc}" + (
+                    f" [reduced to T={T}, V={V} for a profiling capture]"
+                    if (args.rows or args.vocab) else ""),
+                "T_per_gpu": T, "d": d, "V": V, "global_batch": world * T,
+                "vocab_chunk": wl.vocab_chunk or 16384,
+                "parallelism": f"dp{world} (one batch per GPU, no collective on the data path)",
+                "l2": "inputs larger than L2 (W alone is %.2f GB)" % (V * d * 2 / 1e9),
+            },
+            "credited_roofline": {
+                "flops_per_step": credited,
+                "tflops_per_gpu": round(credited / (ms_max / 1e3) / 1e12, 1),
+                "frac_of_bf16_burst": round(credited / (ms_max / 1e3) / 1e12 / peaks["bf16_burst"], 4),
+                "frac_of_bf16_sustained": round(
+                    credited / (ms_max / 1e3) / 1e12 / peaks["bf16_sustained"], 4),
+                "executed_flops_per_step": executed,
+                "note": "credited 4TdV forward (two GEMM passes) + 6TdV backward; the forward "
+                        "runs one GEMM pass and resolves on stored fp32 logits",
+            },
+            "roofline": roof,
+            "kernel_ms_per_step": per_kernel,
+            "e2e": {"value": round(world * T / (e2e_ms / 1e3), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_all,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            n_rows = args.cpu_rows
+            times = time_oracle(data, n_rows, steps=1, warmup=0)
+            out["cpu_baseline"] = {
+                "value": round(n_rows / times[0], 3), "unit": UNIT, "cores": _blas_threads(),
+                "kind": "oracle",
+                "sample": f"{n_rows} of {T} rows (full V, d), float64 forward+backward "
+                          f"in {times[0]:.1f} s; tokens/s = rows / time (linear in rows)",
+            }
+    return out
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = workloads.WORKLOADS[args.workload]
+    data = workloads.make(args.workload)
+    n_rows = args.ref_rows
+    times = time_oracle(data, n_rows, steps=args.steps, warmup=args.warmup)
+    ms = 1e3 * statistics.mean(times)
+    value = n_rows / (ms / 1e3)
+    cores = _blas_threads()
+    sample = (f"{n_rows} of {wl.T} rows (full V={wl.V}, d={wl.d}) per step, float64 "
+              "forward+backward; tokens/s = rows / step time")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name}: {wl.desc}", "T_per_gpu": wl.T, "d": wl.d, "V": wl.V,
+                   "global_batch": wl.T, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=32, help="oracle rows for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=4, help="oracle rows per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="override T (small profiling captures only; not a bench line)")
+    ap.add_argument("--vocab", type=int, default=None,
+                    help="override V (small profiling captures only; not a bench line)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    rank, local_rank, world = dist_env()
+    if world != args.gpus and args.impl == "ours":
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import torch
+            import torch.distributed as dist
+
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(minutes=5),
+                                    device_id=torch.device("cuda", local_rank))
+        try:
+            out = run_ours(args, rank, local_rank, world)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+
+                dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -172,6 +172,31 @@ sts_status sts_get_status(const void* ws, sts_stream_t stream, int64_t* first_ba
 
 const char* sts_status_string(sts_status status);
 
+/* Kernel kinds for the launch counters and the timing facility below. */
+typedef enum {
+  STS_KERNEL_VALIDATE = 0,    /* per-row metadata validation */
+  STS_KERNEL_LOGITS_GEMM = 1, /* forward projection, s = z / tau epilogue */
+  STS_KERNEL_RESOLVE = 2,     /* per-row support resolver */
+  STS_KERNEL_DZ_GEMM = 3,     /* backward recompute, dz epilogue */
+  STS_KERNEL_DW_GEMM = 4,     /* dW slice = dZ^T . H */
+  STS_KERNEL_DH_GEMM = 5,     /* dH (+)= dZ . W slice */
+  STS_KERNEL_KINDS = 6
+} sts_kernel_kind;
+
+/* Number of kernels of a kind this process has launched through the library
+ * (always counted; -1 for an unknown kind). */
+int64_t sts_launch_count(int kind);
+
+/* Host-side timing of every kernel launch (off by default, process-wide).
+ * While on, each launch is bracketed by two CUDA events recorded on the
+ * launch stream; turning it on discards earlier records. Events are host
+ * objects: no device memory is allocated. */
+sts_status sts_timing_enable(int on);
+
+/* Total device time (ms) and launch count of one kind over the records taken
+ * since timing was last turned on. Waits for the recorded events. */
+sts_status sts_timing_read(int kind, double* total_ms, int64_t* launches);
+
 int sts_abi_version(void);
 
 #ifdef __cplusplus

@@ -34,6 +34,10 @@ __all__ = [
     "sts_get_status",
     "sts_status_string",
     "sts_probe_mass_exp",
+    "sts_launch_count",
+    "sts_timing_enable",
+    "sts_timing_read",
+    "KERNEL_KINDS",
     "ROW_TARGET_IN_SUPPORT",
     "ROW_INVALID",
     "ROW_IDENTITY",
@@ -52,6 +56,8 @@ ROW_TARGET_IN_SUPPORT = 1
 ROW_INVALID = 2
 ROW_IDENTITY = 4
 
+KERNEL_KINDS = ("validate", "logits_gemm", "resolve", "dz_gemm", "dw_gemm", "dh_gemm")
+
 EXPORTED_SYMBOLS = (
     "sts_workspace_bytes",
     "sts_forward",
@@ -63,6 +69,9 @@ EXPORTED_SYMBOLS = (
     "sts_status_string",
     "sts_abi_version",
     "sts_probe_mass_exp",
+    "sts_launch_count",
+    "sts_timing_enable",
+    "sts_timing_read",
 )
 
 
@@ -128,6 +137,13 @@ def load():
     lib.sts_status_string.restype = ctypes.c_char_p
     lib.sts_probe_mass_exp.argtypes = [P, ctypes.c_float, P, P, I64, P]
     lib.sts_probe_mass_exp.restype = ctypes.c_int
+    lib.sts_launch_count.argtypes = [ctypes.c_int]
+    lib.sts_launch_count.restype = ctypes.c_int64
+    lib.sts_timing_enable.argtypes = [ctypes.c_int]
+    lib.sts_timing_enable.restype = ctypes.c_int
+    lib.sts_timing_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
+                                    ctypes.POINTER(ctypes.c_int64)]
+    lib.sts_timing_read.restype = ctypes.c_int
     lib.sts_abi_version.argtypes = []
     lib.sts_abi_version.restype = ctypes.c_int
     _lib = lib
@@ -249,7 +265,8 @@ def sts_forward(H, W, target, temperature, top_k, top_p, min_p, *, row_chunk=0, 
 
 
 def sts_backward(H, W, target, temperature, top_k, top_p, min_p, saved, grad_logprob, *,
-                 dW=None, accumulate_dW=False, vocab_chunk=0, ws=None, stream=None, check=False):
+                 dW=None, dH=None, accumulate_dW=False, vocab_chunk=0, ws=None, stream=None,
+                 check=False):
     """dH [T, d] and dW [V, d] (fp32) of sum_t g_t * logprob_t."""
     lib = load()
     T, d, V = _hw(H, W)
@@ -258,7 +275,10 @@ def sts_backward(H, W, target, temperature, top_k, top_p, min_p, saved, grad_log
     sh = _shape(T, d, V, vocab_chunk, 0)
     dev = H.device
     ws = _workspace(sts_workspace_bytes(T, d, V, 1, vocab_chunk, 0), dev, ws)
-    dH = torch.empty((T, d), dtype=torch.float32, device=dev)
+    if dH is None:
+        dH = torch.empty((T, d), dtype=torch.float32, device=dev)
+    else:
+        _need(dH, torch.float32, "dH", (T, d))
     if dW is None:
         if accumulate_dW:
             raise StsError(STS_ERR_NULL, "accumulate_dW needs a dW tensor")
@@ -347,6 +367,30 @@ def sts_probe_mass_exp(s, m, *, stream=None):
     _check(lib.sts_probe_mass_exp(_ptr(s), float(m), _ptr(mass), _ptr(ref), n, _stream(stream)),
            "sts_probe_mass_exp")
     return mass, ref
+
+
+def sts_launch_count(kind=None):
+    """Kernels launched by the library in this process (one kind, or all)."""
+    lib = load()
+    if kind is None:
+        return sum(int(lib.sts_launch_count(i)) for i in range(len(KERNEL_KINDS)))
+    return int(lib.sts_launch_count(KERNEL_KINDS.index(kind) if isinstance(kind, str) else kind))
+
+
+def sts_timing_enable(on=True):
+    _check(load().sts_timing_enable(1 if on else 0), "sts_timing_enable")
+
+
+def sts_timing_read():
+    """{kind: (total_ms, launches)} over the records since timing was enabled."""
+    lib = load()
+    out = {}
+    for i, name in enumerate(KERNEL_KINDS):
+        ms = ctypes.c_double(0.0)
+        n = ctypes.c_int64(0)
+        _check(lib.sts_timing_read(i, ctypes.byref(ms), ctypes.byref(n)), "sts_timing_read")
+        out[name] = (float(ms.value), int(n.value))
+    return out
 
 
 def sts_get_status(ws, stream=None, raise_on_error=False):

@@ -11,8 +11,10 @@
 // PR 74: "What this PR does", item 2, chunked core with a recompute VJP; the
 // "Self-review pass" single-pass vocabulary-chunked backward with write-once
 // weight-gradient slices.)
+#include <atomic>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "gemm_sm100.cuh"
 #include "sts_internal.h"
@@ -90,6 +92,54 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorM
   if (grid <= 0) return cudaSuccess;
   kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(a, b, c, p);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- launch accounting
+
+std::atomic<long long> g_launches[STS_KERNEL_KINDS];
+
+struct TimingState {
+  std::mutex mu;
+  bool on = false;
+  struct Rec {
+    int kind;
+    cudaEvent_t beg, end;
+  };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  cudaEvent_t get() {
+    if (used < pool.size()) return pool[used++];
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    pool.push_back(e);
+    ++used;
+    return e;
+  }
+};
+TimingState g_timing;
+
+// Brackets one kernel launch: counts it and, when timing is on, records the
+// two events around it on the launch stream.
+template <typename F>
+cudaError_t timed_launch(int kind, cudaStream_t st, F&& launch) {
+  g_launches[kind].fetch_add(1, std::memory_order_relaxed);
+  cudaEvent_t b = nullptr, e = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    if (g_timing.on) {
+      b = g_timing.get();
+      e = g_timing.get();
+    }
+  }
+  if (b) cudaEventRecord(b, st);
+  const cudaError_t err = launch();
+  if (e) {
+    cudaEventRecord(e, st);
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    g_timing.recs.push_back({kind, b, e});
+  }
+  return err;
 }
 
 struct DeviceInfo {
@@ -242,8 +292,10 @@ sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, co
   const int np = (int)n_parts(shape);
 
   STS_TRY(reset_header(ws, st));
-  launch_validate(rows->target, rows->temperature, rows->top_p, rows->min_p, T, V, flags, hdr, fwd, st);
-  STS_CUDA(cudaGetLastError());
+  STS_CUDA(timed_launch(STS_KERNEL_VALIDATE, st, [&] {
+    launch_validate(rows->target, rows->temperature, rows->top_p, rows->min_p, T, V, flags, hdr, fwd, st);
+    return cudaGetLastError();
+  }));
 
   CUtensorMap ma, mb;
   if (!map_kmajor(&ma, H, d, T, d, GEMM_BM) || !map_kmajor(&mb, W, d, V, d, GEMM_BN))
@@ -262,7 +314,9 @@ sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, co
     p.err = &hdr->err;
     p.max_part = max_part;
     p.max_ld = np;
-    STS_CUDA((run_gemm<false, false, kEpiLogits>(ma, mb, mc, p, dev.sms, st)));
+    STS_CUDA(timed_launch(STS_KERNEL_LOGITS_GEMM, st, [&] {
+      return run_gemm<false, false, kEpiLogits>(ma, mb, mc, p, dev.sms, st);
+    }));
 
     ResolveArgs a{};
     a.S = S;
@@ -291,7 +345,7 @@ sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, co
     a.row_base = t0;
     a.max_part = max_part;
     a.n_parts = np;
-    STS_CUDA(launch_resolve(a, dev.sms, st));
+    STS_CUDA(timed_launch(STS_KERNEL_RESOLVE, st, [&] { return launch_resolve(a, dev.sms, st); }));
   }
   return STS_OK;
 }
@@ -399,7 +453,9 @@ sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, co
     p.flags = saved->flags;
     p.col_base = (int)v0;
     p.err = &hdr->err;
-    STS_CUDA((run_gemm<false, false, kEpiDZ>(m_h_k, m_w_k, m_dz_out, p, dev.sms, st)));
+    STS_CUDA(timed_launch(STS_KERNEL_DZ_GEMM, st, [&] {
+      return run_gemm<false, false, kEpiDZ>(m_h_k, m_w_k, m_dz_out, p, dev.sms, st);
+    }));
 
     // 2. dW[v0:v0+w] = dZ^T . H (both operands MN-major), written once
     GemmParams q{};
@@ -408,10 +464,10 @@ sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, co
     q.K = (int)T;
     q.c_y0 = (int)v0;
     q.err = &hdr->err;
-    if (accumulate_dW)
-      STS_CUDA((run_gemm<true, true, kEpiReduceF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st)));
-    else
-      STS_CUDA((run_gemm<true, true, kEpiStoreF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st)));
+    STS_CUDA(timed_launch(STS_KERNEL_DW_GEMM, st, [&] {
+      return accumulate_dW ? run_gemm<true, true, kEpiReduceF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st)
+                           : run_gemm<true, true, kEpiStoreF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st);
+    }));
 
     // 3. dH (+)= dZ . W[v0:v0+w] (W read MN-major)
     GemmParams r{};
@@ -420,10 +476,10 @@ sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, co
     r.K = (int)w;
     r.b_k0 = (int)v0;
     r.err = &hdr->err;
-    if (v0 == 0)
-      STS_CUDA((run_gemm<false, true, kEpiStoreF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st)));
-    else
-      STS_CUDA((run_gemm<false, true, kEpiReduceF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st)));
+    STS_CUDA(timed_launch(STS_KERNEL_DH_GEMM, st, [&] {
+      return v0 == 0 ? run_gemm<false, true, kEpiStoreF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st)
+                     : run_gemm<false, true, kEpiReduceF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st);
+    }));
   }
   return STS_OK;
 }
@@ -444,8 +500,10 @@ sts_status sts_filter_logits(const sts_shape* shape, const float* S, const sts_r
   WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
   int32_t* flags = reinterpret_cast<int32_t*>(wsb + sizeof(WsHeader));
   STS_TRY(reset_header(ws, st));
-  launch_validate(nullptr, nullptr, rows->top_p, rows->min_p, shape->T, shape->V, flags, hdr, false, st);
-  STS_CUDA(cudaGetLastError());
+  STS_CUDA(timed_launch(STS_KERNEL_VALIDATE, st, [&] {
+    launch_validate(nullptr, nullptr, rows->top_p, rows->min_p, shape->T, shape->V, flags, hdr, false, st);
+    return cudaGetLastError();
+  }));
   ResolveArgs a{};
   a.S = S;
   a.ld = shape->V;
@@ -462,7 +520,7 @@ sts_status sts_filter_logits(const sts_shape* shape, const float* S, const sts_r
   a.cut_id = cut_id;
   a.mask = mask;
   a.hdr = hdr;
-  STS_CUDA(launch_resolve(a, dev.sms, st));
+  STS_CUDA(timed_launch(STS_KERNEL_RESOLVE, st, [&] { return launch_resolve(a, dev.sms, st); }));
   return STS_OK;
 }
 
@@ -491,7 +549,41 @@ sts_status sts_scaled_logits(const sts_shape* shape, const void* H, const void* 
   p.b_mn0 = (int)v0;
   p.tau = temperature + t0;
   p.err = nullptr;  // no workspace: a bounded-wait timeout here is not reported
-  STS_CUDA((run_gemm<false, false, kEpiLogits>(ma, mb, mc, p, dev.sms, st)));
+  STS_CUDA(timed_launch(STS_KERNEL_LOGITS_GEMM, st, [&] {
+    return run_gemm<false, false, kEpiLogits>(ma, mb, mc, p, dev.sms, st);
+  }));
+  return STS_OK;
+}
+
+int64_t sts_launch_count(int kind) {
+  if (kind < 0 || kind >= STS_KERNEL_KINDS) return -1;
+  return (int64_t)g_launches[kind].load();
+}
+
+sts_status sts_timing_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  g_timing.on = on != 0;
+  g_timing.recs.clear();
+  g_timing.used = 0;
+  return STS_OK;
+}
+
+sts_status sts_timing_read(int kind, double* total_ms, int64_t* launches) {
+  if (kind < 0 || kind >= STS_KERNEL_KINDS) return STS_ERR_SHAPE;
+  if (!total_ms || !launches) return STS_ERR_NULL;
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  double tot = 0.0;
+  int64_t n = 0;
+  for (const auto& r : g_timing.recs) {
+    if (r.kind != kind) continue;
+    if (cudaEventSynchronize(r.end) != cudaSuccess) return STS_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.beg, r.end) != cudaSuccess) return STS_ERR_CUDA;
+    tot += ms;
+    ++n;
+  }
+  *total_ms = tot;
+  *launches = n;
   return STS_OK;
 }
 

@@ -1,0 +1,92 @@
+"""Host-side logic of bench.py without a GPU: clock parsing and rejection,
+max/sum over ranks with a 2-process gloo group, and the reference arm."""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_parse_clock_lines_and_rejection():
+    text = "\n".join([
+        "1800, 1965, 900.1, Not Active, Not Active, Not Active, Active",
+        "1327, 1965, 997.0, Not Active, Not Active, Not Active, Active",
+        "1400, 1965, 990.0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ])
+    clk = bench.parse_clock_lines(text)
+    assert clk["sm_mhz"] == 1400 and clk["sm_max_mhz"] == 1965 and clk["samples"] == 3
+    assert clk["reasons"] == ["sw_power_cap"]
+    assert not bench.clocks_rejected(clk)
+    hot = bench.parse_clock_lines("1500, 1965, 1000, Not Active, Active, Not Active, Not Active")
+    assert bench.clocks_rejected(hot)
+    locked = bench.parse_clock_lines("700, 1965, 400, Not Active, Not Active, Not Active, Not Active")
+    assert bench.clocks_rejected(locked)
+    assert bench.parse_clock_lines("") is None
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mx = bench.reduce_max(10.0 + rank, torch.device("cpu"))
+        sm = bench.reduce_sum(1.5 * (rank + 1), torch.device("cpu"))
+        bench.barrier()
+        q.put((rank, mx, sm))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(2))
+    assert got == [(0, 11.0, 4.5), (1, 11.0, 4.5)]
+
+
+def test_reduce_without_group_is_identity():
+    assert bench.reduce_max(3.5, torch.device("cpu")) == 3.5
+
+
+def test_reference_arm_only_on_rank_zero():
+    class A:
+        workload = 1
+        steps = 1
+        warmup = 0
+        ref_rows = 2
+    assert bench.run_reference(A(), rank=1, world=2) is None
+
+
+def test_reference_arm_json_line():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "1", "--steps", "2", "--warmup", "1"],
+                         capture_output=True, text=True, env=env, timeout=300)
+    assert res.returncode == 0, res.stderr
+    line = json.loads(res.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0

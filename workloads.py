@@ -94,42 +94,11 @@ def _thirds(rng, T):
     return perm[:a], perm[a:2 * a], perm[2 * a:]
 
 
-def make(index: int, T: int | None = None, with_weights: bool = True):
-    """Draw workload ``index`` (1..5). ``T`` overrides the row count (the
-    per-row distributions are unchanged) for reduced-size test cases.
-
-    Returns a dict with ``H`` (uint16 [T, d]), ``W`` (uint16 [V, d], or None
-    when ``with_weights`` is false), ``temperature`` (f32), ``top_k`` (i32),
-    ``top_p`` (f32), ``min_p`` (f32), ``u`` (f64) and ``g`` (f32), plus the
-    ``workload`` record.
-    """
-    wl = WORKLOADS[index]
-    T = wl.T if T is None else int(T)
-    d, V = wl.d, wl.V
-    rng = np.random.Generator(np.random.PCG64(1000 + index))
-
-    H = _normal_bf16(rng, T, d, 1.0)
-    W = None
-    if with_weights:
-        W = _normal_bf16(rng, V, d, 1.0 / np.sqrt(d))
-    else:
-        # keep the stream position identical whether or not W is materialised
-        total = V * d
-        for lo in range(0, total, _CHUNK):
-            rng.standard_normal(min(total, lo + _CHUNK) - lo, dtype=np.float32)
-    if index == 5:
-        n_dup = int(round(0.05 * V))
-        dst = np.sort(rng.choice(np.arange(1, V), size=n_dup, replace=False))
-        src = np.array([rng.integers(0, i) for i in dst], dtype=np.int64)
-        if W is not None:
-            for i, j in zip(dst, src):
-                W[i] = W[j]
-    else:
-        dst = src = np.zeros(0, dtype=np.int64)
-
-    top_k = np.zeros(T, dtype=np.int32)
-    top_p = np.ones(T, dtype=np.float32)
-    min_p = np.zeros(T, dtype=np.float32)
+def _redraw_rows(index, rng, T, V, top_k, top_p, min_p):
+    """Fill the per-row metadata arrays in place; return the temperatures."""
+    top_k[:] = 0
+    top_p[:] = 1.0
+    min_p[:] = 0.0
     if index == 1:
         tau = rng.uniform(0.5, 1.5, T).astype(np.float32)
         top_k[:] = np.where(rng.integers(0, 2, T) == 1, 50, 0)
@@ -158,8 +127,61 @@ def make(index: int, T: int | None = None, with_weights: bool = True):
         top_p[:] = np.where(rng.integers(0, 2, T) == 1, np.float32(0.5), np.float32(1.0))
     else:
         raise ValueError(f"unknown workload {index}")
+    return tau
 
-    u = rng.random(T)
+
+
+def make(index: int, T: int | None = None, with_weights: bool = True, batch: int = 0,
+         V: int | None = None):
+    """Draw workload ``index`` (1..5). ``T`` overrides the row count (the
+    per-row distributions are unchanged) for reduced-size test cases.
+    ``batch`` > 0 draws another batch of rows (H, metadata, u) from a second
+    generator seeded (1000 + index, batch) while W stays the workload's own --
+    one batch per data-parallel rank. ``V`` overrides the vocabulary size
+    (reduced cases for profiling captures only).
+
+    Returns a dict with ``H`` (uint16 [T, d]), ``W`` (uint16 [V, d], or None
+    when ``with_weights`` is false), ``temperature`` (f32), ``top_k`` (i32),
+    ``top_p`` (f32), ``min_p`` (f32), ``u`` (f64) and ``g`` (f32), plus the
+    ``workload`` record.
+    """
+    wl = WORKLOADS[index]
+    T = wl.T if T is None else int(T)
+    d = wl.d
+    V = wl.V if V is None else int(V)
+    rng = np.random.Generator(np.random.PCG64(1000 + index))
+
+    H = _normal_bf16(rng, T, d, 1.0)
+    W = None
+    if with_weights:
+        W = _normal_bf16(rng, V, d, 1.0 / np.sqrt(d))
+    else:
+        # keep the stream position identical whether or not W is materialised
+        total = V * d
+        for lo in range(0, total, _CHUNK):
+            rng.standard_normal(min(total, lo + _CHUNK) - lo, dtype=np.float32)
+    if index == 5:
+        n_dup = int(round(0.05 * V))
+        dst = np.sort(rng.choice(np.arange(1, V), size=n_dup, replace=False))
+        src = np.array([rng.integers(0, i) for i in dst], dtype=np.int64)
+        if W is not None:
+            for i, j in zip(dst, src):
+                W[i] = W[j]
+    else:
+        dst = src = np.zeros(0, dtype=np.int64)
+
+    top_k = np.zeros(T, dtype=np.int32)
+    top_p = np.ones(T, dtype=np.float32)
+    min_p = np.zeros(T, dtype=np.float32)
+    tau = _redraw_rows(index, rng, T, V, top_k, top_p, min_p)
+
+    if batch:
+        rng_b = np.random.Generator(np.random.PCG64([1000 + index, int(batch)]))
+        H = _normal_bf16(rng_b, T, d, 1.0)
+        tau = _redraw_rows(index, rng_b, T, V, top_k, top_p, min_p)
+        u = rng_b.random(T)
+    else:
+        u = rng.random(T)
     g = np.ones(T, dtype=np.float32)
     return {
         "workload": wl,
