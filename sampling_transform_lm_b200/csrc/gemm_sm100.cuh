@@ -22,7 +22,10 @@
 //   kEpiLogits    s = z / tau_row (IEEE fp32 division) -> fp32
 //   kEpiDZ        s = z / tau_row; p = exp(s - LSE_S) on the support, 0 off it;
 //                 dz = g/tau * (1[col == y] - p) (0 for rows whose target is
-//                 out of support or invalid) -> bf16
+//                 out of support or invalid) -> bf16. Support membership uses
+//                 the forward's exact quotient (re-divided near the cut); p
+//                 uses z * (1/tau) and the hardware exp2 (relative error
+//                 ~2e-6, well below the bf16 rounding of dz)
 //   kEpiStoreF32  acc -> fp32
 //   kEpiReduceF32 acc -> fp32, added in place (TMA reduce-add)
 #pragma once
@@ -255,7 +258,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const bool row_ok = row < p.M;
       const bool quarter_live = row0 < p.M;
 
-      float tau = 1.f, lse = 0.f, cut = 0.f, coef = 0.f;
+      float tau = 1.f, lse = 0.f, cut = 0.f, coef = 0.f, rtau = 1.f, cut_lo = 0.f, cut_hi = 0.f;
       int cut_id = -1;
       long long y = -1;
       if (EPI == kEpiLogits || EPI == kEpiDZ) {
@@ -271,6 +274,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             cut_id = p.cut_id[row];
             y = p.target[row];
             coef = __fdiv_rn(p.grad[row], tau);
+            rtau = __frcp_rn(tau);
+            const float margin = fabsf(cut) * 1e-6f + 1e-30f;  // ~8 ulp of the cut
+            cut_lo = cut - margin;
+            cut_hi = cut + margin;
           }
         }
       }
@@ -307,10 +314,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const long long col0 = (long long)p.col_base + ncol0;
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
-              const float s = __fdiv_rn(v[j], tau);
+              // z * (1/tau) is within 2 ulp of the forward's IEEE quotient; only
+              // values that close to the cut are re-divided exactly, so the
+              // membership decision is the forward's bit for bit
+              float sf = v[j] * rtau;
               const long long col = col0 + j;
-              const bool member = (s > cut) || (s == cut && col <= (long long)cut_id);
-              const float pr = member ? expf(s - lse) : 0.f;
+              bool member = sf > cut_hi;
+              if (!member && sf >= cut_lo) {
+                sf = __fdiv_rn(v[j], tau);
+                member = (sf > cut) || (sf == cut && col <= (long long)cut_id);
+              }
+              const float pr = member ? __expf(sf - lse) : 0.f;
               v[j] = coef * ((col == y ? 1.f : 0.f) - pr);
             }
           } else {

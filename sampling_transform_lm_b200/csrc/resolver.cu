@@ -48,7 +48,7 @@ namespace {
 constexpr int RT = 512;             // threads per resolver CTA
 constexpr int NWARP = RT / 32;
 constexpr int NB = 4096;            // histogram buckets per level
-constexpr int CAP = 4096;           // candidate buffer (composite keys)
+constexpr int CAP = 8192;           // candidate buffer (composite keys)
 constexpr float BIN_SCALE = 128.f;  // level-0 buckets per logit unit
 constexpr int MAX_LEVELS = 8;
 constexpr int UNROLL = 4;           // float4 loads in flight per thread
@@ -57,9 +57,10 @@ struct RSmem {
   double mass[NB];
   double tab[NB];  // exp(-b / 128)
   unsigned long long cand[CAP];
-  double cq[CAP];
+  double cq[CAP / 2];  // inclusive mass scan of at most CAP / 2 sorted candidates
   int cnt[NB];
   double red_d[NWARP];
+  double red_m[NWARP * 8 + 8];
   unsigned long long red_u[NWARP];
   long long red_l[NWARP];
   float red_f[NWARP];
@@ -67,6 +68,7 @@ struct RSmem {
   long long bl[4];
   int bi[4];
   int ncand;
+  int wcount[NWARP];  // fast path: fill level of each warp's gather slice
 };
 
 // ---------------------------------------------------------------- keys
@@ -119,6 +121,22 @@ __device__ __forceinline__ double qmass(const RSmem& sm, float s, float m) {
 
 // ---------------------------------------------------------------- streaming
 
+// Read-only streaming loads that do not allocate in L1 (most of the SM's
+// on-chip memory is shared memory here, so L1 is small).
+__device__ __forceinline__ float4 ld_stream4(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float ld_stream(const float* p) {
+  float v;
+  asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+
 // Apply f(value, index) to every element of the row. VEC: the row start is
 // 16-byte aligned, so UNROLL float4 loads per thread are kept in flight.
 template <bool VEC, typename F>
@@ -131,7 +149,7 @@ __device__ __forceinline__ void for_each(const float* __restrict__ x, int V, F&&
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
         const int i = base + u * RT + (int)threadIdx.x;
-        if (i < V4) v[u] = x4[i];
+        if (i < V4) v[u] = ld_stream4(x4 + i);
       }
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
@@ -144,7 +162,7 @@ __device__ __forceinline__ void for_each(const float* __restrict__ x, int V, F&&
         }
       }
     }
-    for (int i = 4 * V4 + (int)threadIdx.x; i < V; i += RT) f(x[i], i);
+    for (int i = 4 * V4 + (int)threadIdx.x; i < V; i += RT) f(ld_stream(x + i), i);
   } else {
     constexpr int U = 4 * UNROLL;
     for (int base = 0; base < V; base += RT * U) {
@@ -152,7 +170,7 @@ __device__ __forceinline__ void for_each(const float* __restrict__ x, int V, F&&
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int i = base + u * RT + (int)threadIdx.x;
-        if (i < V) v[u] = x[i];
+        if (i < V) v[u] = ld_stream(x + i);
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -212,6 +230,32 @@ __device__ long long block_sum_l(long long v, RSmem& sm) {
   const long long r = sm.red_l[0];
   __syncthreads();
   return r;
+}
+
+// Sums of N doubles over the block in one exchange (two barriers).
+template <int N>
+__device__ void block_sum_multi(double (&v)[N], RSmem& sm) {
+  static_assert(N <= 8, "scratch holds 8 values per warp");
+#pragma unroll
+  for (int k = 0; k < N; ++k)
+    for (int o = 16; o; o >>= 1) v[k] += __shfl_down_sync(0xffffffffu, v[k], o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0)
+#pragma unroll
+    for (int k = 0; k < N; ++k) sm.red_m[w * 8 + k] = v[k];
+  __syncthreads();
+  if (w == 0) {
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
+      double t = l < NWARP ? sm.red_m[l * 8 + k] : 0.0;
+      for (int o = 16; o; o >>= 1) t += __shfl_down_sync(0xffffffffu, t, o);
+      if (l == 0) sm.red_m[NWARP * 8 + k] = t;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < N; ++k) v[k] = sm.red_m[NWARP * 8 + k];
+  __syncthreads();
 }
 
 template <bool kMax>
@@ -339,23 +383,6 @@ __device__ __noinline__ void pick_bucket(RSmem& sm, int crit, long long need, do
   __syncthreads();
 }
 
-// Count and mass of every bucket before bucket b (b may be NB: all buckets).
-__device__ __noinline__ void bucket_prefix(RSmem& sm, int b, long long& cnt_excl, double& mass_excl) {
-  constexpr int PER = NB / RT;
-  const int base = threadIdx.x * PER;
-  long long lc = 0;
-  double lm = 0.0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    if (base + i < b) {
-      lc += sm.cnt[base + i];
-      lm += sm.mass[base + i];
-    }
-  }
-  cnt_excl = block_sum_l(lc, sm);
-  mass_excl = block_sum_d(lm, sm);
-}
-
 // Level-0 histogram of the row (counts and float64 masses per bucket); also
 // the total mass and the last element of the order when asked.
 template <bool VEC>
@@ -385,35 +412,55 @@ __device__ __noinline__ void build_hist0(RSmem& sm, const float* __restrict__ x,
 
 // Sort sm.cand[0..n) descending (composite keys are distinct) and write the
 // inclusive float64 prefix of the masses to sm.cq (thread order, deterministic).
-__device__ __noinline__ void sort_and_scan(RSmem& sm, int n, float m) {
+// Sorts the n (<= CAP / 2) candidates of sm.cand[a0, a0 + n) into
+// sm.cand[0, n) and writes their inclusive mass scan to sm.cq[0, n) (the rest
+// of the candidate buffer is scratch afterwards).
+__device__ __noinline__ void sort_and_scan(RSmem& sm, int a0, int n, float m) {
+  constexpr int PER = (CAP / 2) / RT;
+  n = min(n, CAP / 2);
+  if (a0 != 0) {
+    unsigned long long t[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int j = (int)threadIdx.x * PER + i;
+      t[i] = j < n ? sm.cand[a0 + j] : 0ull;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int j = (int)threadIdx.x * PER + i;
+      if (j < n) sm.cand[j] = t[i];
+    }
+    __syncthreads();
+  }
+  unsigned long long* c = sm.cand;
   int n2 = 2;
   while (n2 < n) n2 <<= 1;
-  for (int i = n + (int)threadIdx.x; i < n2; i += RT) sm.cand[i] = 0ull;  // sorts last
+  for (int i = n + (int)threadIdx.x; i < n2; i += RT) c[i] = 0ull;  // sorts last
   __syncthreads();
   for (int k = 2; k <= n2; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
       for (int i = threadIdx.x; i < n2; i += RT) {
         const int ixj = i ^ j;
         if (ixj > i) {
-          const unsigned long long a = sm.cand[i], c = sm.cand[ixj];
+          const unsigned long long x0 = c[i], x1 = c[ixj];
           const bool desc = (i & k) == 0;
-          if (desc ? (a < c) : (a > c)) {
-            sm.cand[i] = c;
-            sm.cand[ixj] = a;
+          if (desc ? (x0 < x1) : (x0 > x1)) {
+            c[i] = x1;
+            c[ixj] = x0;
           }
         }
       }
       __syncthreads();
     }
   }
-  constexpr int PER = CAP / RT;
   const int base = threadIdx.x * PER;
   double loc[PER];
   double run = 0.0;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int j = base + i;
-    const double qv = j < n ? qmass(sm, ckey_value(sm.cand[j]), m) : 0.0;
+    const double qv = j < n ? qmass(sm, ckey_value(c[j]), m) : 0.0;
     run += qv;
     loc[i] = run;
   }
@@ -440,6 +487,20 @@ __device__ __noinline__ int first_mass_hit(RSmem& sm, int lo, int hi, double bas
   return j;
 }
 
+// Warp-cooperative append: every active lane with `take` set gets a distinct
+// slot from one atomic per warp on *counter (no same-address contention).
+__device__ __forceinline__ int warp_slot(int* counter, bool take) {
+  const unsigned act = __activemask();
+  const unsigned mask = __ballot_sync(act, take);
+  if (mask == 0u) return -1;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(mask) - 1;
+  int base = 0;
+  if (lane == leader) base = atomicAdd(counter, __popc(mask));
+  base = __shfl_sync(act, base, leader);
+  return take ? base + __popc(mask & ((1u << lane) - 1u)) : -1;
+}
+
 // General search: the element of the order where the criterion is first met,
 // refining oversized buckets. Returns false if the refinement bound is hit.
 template <bool VEC>
@@ -459,7 +520,7 @@ __device__ __noinline__ bool locate(RSmem& sm, const float* __restrict__ x, int 
   bool refined = false;
   __syncthreads();
 
-  for (int level = 0; set_cnt > CAP; ++level) {
+  for (int level = 0; set_cnt > CAP / 2; ++level) {
     if (level >= MAX_LEVELS) return false;
     unsigned long long kmin = ~0ull, kmax = 0ull;
     for_each<VEC>(x, V, [&](float s, int i) {
@@ -510,15 +571,14 @@ __device__ __noinline__ bool locate(RSmem& sm, const float* __restrict__ x, int 
   if (threadIdx.x == 0) sm.ncand = 0;
   __syncthreads();
   for_each<VEC>(x, V, [&](float s, int i) {
-    if (bin0(s, m) != b) return;
     const unsigned long long K = ckey(s, i);
-    if (refined && (K < Klo || K > Khi)) return;
-    const int slot = atomicAdd(&sm.ncand, 1);
-    if (slot < CAP) sm.cand[slot] = K;
+    const bool take = bin0(s, m) == b && !(refined && (K < Klo || K > Khi));
+    const int slot = warp_slot(&sm.ncand, take);
+    if (slot >= 0 && slot < CAP) sm.cand[slot] = K;
   });
   __syncthreads();
   const int n = min(sm.ncand, CAP);
-  sort_and_scan(sm, n, m);
+  sort_and_scan(sm, 0, n, m);
   int jstar;
   if (crit == kCount)
     jstar = (int)(need - above_cnt - 1);
@@ -553,14 +613,42 @@ __device__ __noinline__ Cut min_p_cut_pass(RSmem& sm, const float* __restrict__ 
   return cm;
 }
 
-// Smallest fp32 t (as a key) with exp(t - m) >= mu, mu in (0, 1].
+// Smallest fp32 t (as a key) with exp(t - m) >= mu, mu in (0, 1]: start at
+// the fp32 value nearest m + ln(mu), walk a few keys to the boundary, and
+// finish by bisection over fp32 bit patterns if the walk did not close it.
 __device__ __noinline__ uint32_t min_p_threshold_key(float m, float mu) {
-  uint32_t lo = key32(-FLT_MAX), hi = key32(m);  // P(lo) false, P(hi) true
   const double md = (double)m, mud = (double)mu;
+  auto keep = [&](uint32_t k) { return exp((double)key32_value(k) - md) >= mud; };
+  uint32_t lo = key32(-FLT_MAX), hi = key32(m);  // keep(lo) false, keep(hi) true
   if (exp((double)(-FLT_MAX) - md) >= mud) return lo;
+  const double t0 = md + log(mud);
+  uint32_t k0 = key32(t0 > -FLT_MAX ? (float)t0 : -FLT_MAX);
+  if (k0 <= lo) k0 = lo + 1;
+  if (k0 > hi) k0 = hi;
+  if (keep(k0)) {
+    hi = k0;
+    for (int i = 0; i < 8 && hi - lo > 1; ++i) {
+      if (keep(hi - 1)) {
+        --hi;
+      } else {
+        lo = hi - 1;
+        break;
+      }
+    }
+  } else {
+    lo = k0;
+    for (int i = 0; i < 8 && hi - lo > 1; ++i) {
+      if (!keep(lo + 1)) {
+        ++lo;
+      } else {
+        hi = lo + 1;
+        break;
+      }
+    }
+  }
   while (hi - lo > 1u) {
     const uint32_t mid = lo + (hi - lo) / 2u;
-    if (exp((double)key32_value(mid) - md) >= mud)
+    if (keep(mid))
       hi = mid;
     else
       lo = mid;
@@ -575,47 +663,468 @@ __device__ __noinline__ float row_max_pass(const float* __restrict__ x, int V) {
   return lm;
 }
 
-// Gather every element of buckets [0, bk] into sm.cand; returns the count.
-template <bool VEC>
-__device__ __noinline__ int gather_prefix(RSmem& sm, const float* __restrict__ x, int V, float m,
-                                          int bk) {
-  if (threadIdx.x == 0) sm.ncand = 0;
-  __syncthreads();
-  for_each<VEC>(x, V, [&](float s, int i) {
-    if (bin0(s, m) > bk) return;
-    const int slot = atomicAdd(&sm.ncand, 1);
-    if (slot < CAP) sm.cand[slot] = ckey(s, i);
-  });
-  __syncthreads();
-  const int n = min(sm.ncand, CAP);
-  __syncthreads();
-  return n;
-}
 
 // Gather the elements of buckets bp and bm (either may be -1) into sm.cand
 // and, when kt is live, return the last element with key >= kt among the
-// buckets up to bm (the end of the min-p prefix).
+
+// ---------------------------------------------------------------- exact path
+// Float64 mass histogram (atomics) and the general search: used when the fast
+// path below cannot prove its window holds the cut (large top-k, oversized
+// buckets, a crossing outside the estimated window).
 template <bool VEC>
-__device__ __noinline__ int gather_two(RSmem& sm, const float* __restrict__ x, int V, float m,
-                                       int bp, int bm, bool mu_on, uint32_t kt,
-                                       unsigned long long* K_mu) {
-  if (threadIdx.x == 0) sm.ncand = 0;
+__device__ __noinline__ bool resolve_row_exact(RSmem& sm, const float* __restrict__ x, int V,
+                                               float m, int k, float p, float mu, uint32_t kt,
+                                               bool& hist_valid, Cut& best) {
+  const bool k_on = k >= 1 && k < V, p_on = p < 1.0f, mu_on = mu > 0.0f;
+  double Z;
+  unsigned long long Klast;
+  build_hist0<VEC>(sm, x, V, m, &Z, &Klast);
+  hist_valid = true;
+  best = Cut{Klast, (long long)V, Z};
+  double Zk = Z;
+  if (k_on) {
+    Cut ck;
+    if (!locate<VEC>(sm, x, V, m, hist_valid, kCount, (long long)k, 0.0, ck)) return false;
+    Zk = ck.mass;
+    take_earlier(best, ck);
+  }
+  if (p_on) {
+    Cut cp;
+    if (!locate<VEC>(sm, x, V, m, hist_valid, kMassGE, 0, (double)p * Zk, cp)) return false;
+    take_earlier(best, cp);
+  }
+  if (mu_on) take_earlier(best, min_p_cut_pass<VEC>(sm, x, V, m, kt));
+  return true;
+}
+
+// ---------------------------------------------------------------- fast path
+
+// Count-only level-0 histogram.
+template <bool VEC>
+__device__ __noinline__ void count_hist(RSmem& sm, const float* __restrict__ x, int V, float m) {
+  for (int i = threadIdx.x; i < NB; i += RT) sm.cnt[i] = 0;
   __syncthreads();
+  for_each<VEC>(x, V, [&](float s, int) { atomicAdd(&sm.cnt[bin0(s, m)], 1); });
+  __syncthreads();
+}
+
+// Sum of counts over buckets [lo, hi).
+__device__ long long count_range(RSmem& sm, int lo, int hi) {
+  long long c = 0;
+  for (int i = lo + (int)threadIdx.x; i < hi; i += RT) c += sm.cnt[i];
+  return block_sum_l(c, sm);
+}
+
+struct Pass2 {
+  // plan
+  bool need_z;       // exact total mass (and mass before w_lo / b_mu) for every element
+  bool need_last;    // last element of the order
+  int w_lo, w_hi;    // window of buckets gathered by bucket into regions (w_lo > w_hi: none)
+  int woff[3];       // region offsets in sm.cand of the window buckets
+  int b_mu;          // min-p boundary bucket (-1: min-p off)
+  uint32_t kt;       // min-p threshold key
+  int bk;            // gather every bucket <= bk into sm.cand (-1: no prefix gather)
+  // results
+  double z, a_p, a_mu;
+  unsigned long long k_last;
+  bool overflow;     // a warp's gather slice overflowed
+};
+
+// Plan of pass 2, passed by value so every field lives in a register.
+struct Plan2 {
+  int need_last;            // last element of the order (per-thread key minimum)
+  int g_lo, g_hi;           // gather buckets [g_lo, g_hi] ...
+  int g2_lo, g2_hi;         // ... and [g2_lo, g2_hi] (empty ranges: lo > hi)
+  int w_lo;                 // mass before w_lo is accumulated (a_p)
+  int b_mu;                 // mass before b_mu is accumulated (a_mu); -1: off
+};
+
+constexpr int WCAP = CAP / NWARP;  // private gather slots per warp
+
+// One pass over the row: exact float64 masses accumulated in registers, and
+// the elements of up to two bucket ranges gathered into per-warp slices of
+// sm.cand with a warp-uniform fill level (ballot + popc: no shared counters).
+// The mass polynomial of E consecutive elements is evaluated as independent
+// chains and summed into split accumulators, so float64 latency is covered.
+// Every lane of a warp runs every batch (invalid slots masked), so the warp
+// votes always see the full warp.
+template <bool VEC, bool NEED_Z>
+__device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, int V, float m,
+                                        const Plan2 pl, Pass2& P) {
+  constexpr int E = 8;
+  const double md = (double)m;
+  const bool need_last = pl.need_last != 0;
+  const int g_lo = pl.g_lo, g_hi = pl.g_hi, g2_lo = pl.g2_lo, g2_hi = pl.g2_hi;
+  const int w_lo = pl.w_lo, b_mu = pl.b_mu;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  unsigned long long* wbuf = sm.cand + warp * WCAP;
+  int wfill = 0;  // warp-uniform
+  double z[2] = {0.0, 0.0}, ap[2] = {0.0, 0.0}, amu[2] = {0.0, 0.0};
   unsigned long long kl = ~0ull;
-  for_each<VEC>(x, V, [&](float s, int i) {
-    const int b0 = bin0(s, m);
-    if (mu_on && b0 <= bm && key32(s) >= kt) {
-      const unsigned long long K = ckey(s, i);
-      kl = K < kl ? K : kl;
+
+  auto batch = [&](const float (&sv)[E], int i0, int nvalid) {
+    int bb[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) bb[e] = bin0(sv[e], m);
+    if (NEED_Z) {
+      double qq[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const double xx = (double)sv[e] - md;
+        const double r = fma((double)bb[e], 1.0 / 128.0, xx);
+        double p = 1.0 / 720.0;
+        p = fma(p, r, 1.0 / 120.0);
+        p = fma(p, r, 1.0 / 24.0);
+        p = fma(p, r, 1.0 / 6.0);
+        p = fma(p, r, 0.5);
+        p = fma(p, r, 1.0);
+        p = fma(p, r, 1.0);
+        qq[e] = sm.tab[bb[e]] * p;
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (bb[e] >= NB - 1) qq[e] = exp((double)sv[e] - md);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const double q = e < nvalid ? qq[e] : 0.0;
+        z[e & 1] += q;
+        ap[e & 1] += bb[e] < w_lo ? q : 0.0;
+        amu[e & 1] += bb[e] < b_mu ? q : 0.0;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (e < nvalid && bb[e] < b_mu) amu[e & 1] += qmass_b(sm.tab, sv[e], md, bb[e]);
     }
-    if (b0 != bp && b0 != bm) return;
-    const int slot = atomicAdd(&sm.ncand, 1);
-    if (slot < CAP) sm.cand[slot] = ckey(s, i);
-  });
-  *K_mu = block_ext_u<false>(kl, sm);
-  const int n = min(sm.ncand, CAP);
+    if (need_last) {
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (e < nvalid) {
+          const unsigned long long K = ckey(sv[e], i0 + e);
+          kl = K < kl ? K : kl;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int b = bb[e];
+      const bool g = e < nvalid && ((b >= g_lo && b <= g_hi) || (b >= g2_lo && b <= g2_hi));
+      const unsigned mask = __ballot_sync(0xffffffffu, g);
+      if (mask) {
+        const int slot = wfill + __popc(mask & lt);
+        if (g && slot < WCAP) wbuf[slot] = ckey(sv[e], i0 + e);
+        wfill += __popc(mask);
+      }
+    }
+  };
+
+  if (VEC) {
+    const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
+    const int V8 = V / E;  // batches of 8 consecutive elements (two float4)
+    for (int base = 0; base < V8; base += RT * 2) {
+      float4 va[2], vb[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int i = base + u * RT + (int)threadIdx.x;
+        if (i < V8) {
+          va[u] = ld_stream4(x4 + 2 * i);
+          vb[u] = ld_stream4(x4 + 2 * i + 1);
+        } else {
+          va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll 1
+      for (int u = 0; u < 2; ++u) {
+        const int i = base + u * RT + (int)threadIdx.x;
+        const float sv[E] = {va[u].x, va[u].y, va[u].z, va[u].w, vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+        batch(sv, E * i, i < V8 ? E : 0);
+      }
+    }
+    for (int i0 = E * V8; i0 < V; i0 += RT) {
+      const int i = i0 + (int)threadIdx.x;
+      float sv[E];
+      const float v = i < V ? ld_stream(x + i) : 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) sv[e] = v;
+      batch(sv, i, i < V ? 1 : 0);
+    }
+  } else {
+    for (int i0 = 0; i0 < V; i0 += RT) {
+      const int i = i0 + (int)threadIdx.x;
+      float sv[E];
+      const float v = i < V ? ld_stream(x + i) : 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) sv[e] = v;
+      batch(sv, i, i < V ? 1 : 0);
+    }
+  }
+  if (lane == 0) sm.wcount[warp] = wfill;
+  double sums[3] = {z[0] + z[1], ap[0] + ap[1], amu[0] + amu[1]};
+  block_sum_multi<3>(sums, sm);
+  P.z = sums[0];
+  P.a_p = sums[1];
+  P.a_mu = sums[2];
+  P.k_last = need_last ? block_ext_u<false>(kl, sm) : ~0ull;
+  int ovf = 0;
+  for (int w = 0; w < NWARP; ++w) ovf |= sm.wcount[w] > WCAP ? 1 : 0;
+  P.overflow = ovf != 0;
   __syncthreads();
-  return n;
+}
+
+template <bool VEC>
+__device__ void pass2(RSmem& sm, const float* __restrict__ x, int V, float m, bool need_z,
+                      const Plan2& pl, Pass2& P) {
+  if (need_z)
+    pass2_impl<VEC, true>(sm, x, V, m, pl, P);
+  else
+    pass2_impl<VEC, false>(sm, x, V, m, pl, P);
+}
+
+// Move the gathered candidates whose bucket lies in [lo, hi] from the per-warp
+// slices to sm.cand[0, n) (block scan, order irrelevant: they are sorted
+// next). Returns n.
+__device__ __noinline__ int compact_gathered(RSmem& sm, float m, int lo, int hi) {
+  constexpr int PER = CAP / RT;  // slots per thread (inside one warp slice)
+  unsigned long long t[PER];
+  int mine = 0;
+  const int base = (int)threadIdx.x * PER;
+  const int wcnt = sm.wcount[base / WCAP];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int slot = base + i;
+    const bool ok = (slot % WCAP) < wcnt;
+    const unsigned long long K = ok ? sm.cand[slot] : 0ull;
+    const int b = ok ? bin0(ckey_value(K), m) : -1;
+    t[i] = (ok && b >= lo && b <= hi) ? K : 0ull;
+    mine += t[i] != 0ull ? 1 : 0;
+  }
+  long long tot;
+  const int off = (int)block_exscan<long long>((long long)mine, sm.red_l, tot);
+  // t[] holds this thread's share; the buffer is rewritten from the front
+  int o = off;
+#pragma unroll
+  for (int i = 0; i < PER; ++i)
+    if (t[i] != 0ull) sm.cand[o++] = t[i];
+  __syncthreads();
+  return (int)tot;
+}
+
+// Exact mass and count of the gathered candidates in bucket b, and (for
+// min-p) of those with key >= kt, plus the smallest such key.
+__device__ __noinline__ void gathered_bucket_stats(RSmem& sm, float m, int b, uint32_t kt,
+                                                   double& mass, long long& cnt, double& kept_mass,
+                                                   long long& kept_cnt, unsigned long long& k_min) {
+  constexpr int PER = CAP / RT;
+  const int base = (int)threadIdx.x * PER;
+  const int wcnt = sm.wcount[base / WCAP];
+  double ms = 0.0, km = 0.0;
+  long long c = 0, kc = 0;
+  unsigned long long kmn = ~0ull;
+  for (int i = 0; i < PER; ++i) {
+    const int slot = base + i;
+    if ((slot % WCAP) >= wcnt) continue;
+    const unsigned long long K = sm.cand[slot];
+    const float v = ckey_value(K);
+    if (bin0(v, m) != b) continue;
+    const double q = qmass(sm, v, m);
+    ms += q;
+    ++c;
+    if ((uint32_t)(K >> 32) >= kt) {
+      km += q;
+      ++kc;
+      kmn = K < kmn ? K : kmn;
+    }
+  }
+  mass = block_sum_d(ms, sm);
+  cnt = block_sum_l(c, sm);
+  kept_mass = block_sum_d(km, sm);
+  kept_cnt = block_sum_l(kc, sm);
+  k_min = block_ext_u<false>(kmn, sm);
+}
+
+// Exact masses and counts of the gathered candidates of buckets lo..hi
+// (hi - lo <= 2), in one sweep over the per-warp slices.
+__device__ __noinline__ void window_stats(RSmem& sm, float m, int lo, int hi, double (&wm)[3],
+                                          long long (&wc)[3]) {
+  constexpr int PER = CAP / RT;
+  const int base = (int)threadIdx.x * PER;
+  const int wcnt = sm.wcount[base / WCAP];
+  double ms[3] = {0.0, 0.0, 0.0};
+  long long c[3] = {0, 0, 0};
+  for (int i = 0; i < PER; ++i) {
+    const int slot = base + i;
+    if ((slot % WCAP) >= wcnt) continue;
+    const float v = ckey_value(sm.cand[slot]);
+    const int b = bin0(v, m);
+    if (b < lo || b > hi) continue;
+    const double q = qmass(sm, v, m);
+#pragma unroll
+    for (int w = 0; w < 3; ++w)
+      if (b - lo == w) {
+        ms[w] += q;
+        ++c[w];
+      }
+  }
+  double v[6] = {ms[0], ms[1], ms[2], (double)c[0], (double)c[1], (double)c[2]};
+  block_sum_multi<6>(v, sm);
+#pragma unroll
+  for (int w = 0; w < 3; ++w) {
+    wm[w] = v[w];
+    wc[w] = (long long)v[3 + w];
+  }
+}
+
+// Last non-empty bucket strictly before b (-1 if none).
+__device__ int prev_nonempty(RSmem& sm, int b) {
+  int mine = -1;
+  for (int i = threadIdx.x; i < b; i += RT)
+    if (sm.cnt[i] > 0) mine = i;
+  return (int)block_ext_u<true>((unsigned long long)(mine + 1), sm) - 1;
+}
+
+// Resolve a row with one count pass and one exact pass. Returns false when the
+// exact path must decide instead.
+template <bool VEC>
+__device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict__ x, int V, float m,
+                                              int k, float p, float mu, uint32_t kt, Cut& best) {
+  const bool k_on = k >= 1 && k < V, p_on = p < 1.0f, mu_on = mu > 0.0f;
+  Plan2 pl;
+  pl.need_last = 0;
+  pl.g_lo = 1;
+  pl.g_hi = 0;
+  pl.g2_lo = 1;
+  pl.g2_hi = 0;
+  pl.w_lo = -1;
+  pl.b_mu = -1;
+  Pass2 P;
+
+  if (!k_on && !p_on && !mu_on) {  // identity: total mass and the last element only
+    pl.need_last = 1;
+    pass2<VEC>(sm, x, V, m, true, pl, P);
+    best = Cut{P.k_last, (long long)V, P.z};
+    return true;
+  }
+
+  count_hist<VEC>(sm, x, V, m);
+
+  if (k_on) {
+    // small k: the prefix of buckets up to the k-th element's fits the buffer
+    // and holds every cut that can come before the top-k cut
+    int bk;
+    long long ce;
+    double me;
+    pick_bucket(sm, kCount, (long long)k, 0.0, 0, 0.0, bk, ce, me);
+    const long long incl = ce + sm.cnt[bk];
+    __syncthreads();
+    if (incl > CAP / 2) return false;  // keep the per-warp slices far from full
+    pl.g_lo = 0;
+    pl.g_hi = bk;
+    pass2<VEC>(sm, x, V, m, false, pl, P);
+    if (P.overflow) return false;
+    const int n = compact_gathered(sm, m, 0, bk);
+    sort_and_scan(sm, 0, n, m);
+    const int jk = min(k, n) - 1;
+    Cut ck{sm.cand[jk], (long long)jk + 1, sm.cq[jk]};
+    best = ck;
+    const double Zk = ck.mass;
+    if (p_on) {
+      const int jp = first_mass_hit(sm, 0, jk + 1, 0.0, 0.0, kMassGE, (double)p * Zk);
+      take_earlier(best, Cut{sm.cand[jp], (long long)jp + 1, sm.cq[jp]});
+    }
+    if (mu_on) {
+      int mine = 0;
+      for (int j = threadIdx.x; j < n; j += RT) mine += (uint32_t)(sm.cand[j] >> 32) >= kt ? 1 : 0;
+      const int nk = (int)block_sum_l(mine, sm);
+      if (nk >= 1 && nk < n) take_earlier(best, Cut{sm.cand[nk - 1], (long long)nk, sm.cq[nk - 1]});
+    }
+    __syncthreads();
+    return true;
+  }
+
+  // top-k off: estimate the top-p crossing bucket from counts x mid-bucket
+  // weights and gather a 3-bucket window around it; for min-p gather the
+  // threshold's bucket and the non-empty bucket before it
+  long long before_win = 0, before_mu = 0;
+  int lo = 0, hi = -1, bm = -1, bprev = -1;
+  long long gathered = 0;
+  if (p_on) {
+    for (int i = threadIdx.x; i < NB; i += RT)
+      sm.mass[i] = i < NB - 1 ? (double)sm.cnt[i] * sm.tab[i] * sm.bd[3] : 0.0;
+    __syncthreads();
+    double zl = 0.0;
+    for (int i = threadIdx.x; i < NB; i += RT) zl += sm.mass[i];
+    const double zhat = block_sum_d(zl, sm);
+    int bh;
+    long long ce;
+    double me;
+    pick_bucket(sm, kMassGE, 0, (double)p * zhat, 0, 0.0, bh, ce, me);
+    lo = bh > 0 ? bh - 1 : 0;
+    hi = bh < NB - 1 ? bh + 1 : NB - 1;
+    gathered += count_range(sm, lo, hi + 1);
+    before_win = count_range(sm, 0, lo);
+    pl.g_lo = lo;
+    pl.g_hi = hi;
+    pl.w_lo = lo;
+  }
+  if (mu_on) {
+    bm = bin0(key32_value(kt), m);
+    bprev = prev_nonempty(sm, bm);
+    before_mu = count_range(sm, 0, bm);
+    const int a0 = bprev >= 0 ? bprev : bm;
+    gathered += count_range(sm, a0, bm + 1);
+    pl.g2_lo = a0;
+    pl.g2_hi = bm;
+    pl.b_mu = bm;
+  }
+  __syncthreads();
+  if (gathered > CAP / 2) return false;  // keep the per-warp slices far from full
+  pass2<VEC>(sm, x, V, m, p_on, pl, P);
+  if (P.overflow) return false;
+
+  bool have = false;
+  if (mu_on) {
+    double mass, kmass;
+    long long cnt, kcnt;
+    unsigned long long kmin;
+    gathered_bucket_stats(sm, m, bm, kt, mass, cnt, kmass, kcnt, kmin);
+    if (kcnt == 0 && bprev >= 0) {
+      // nothing of bucket bm is kept: the min-p prefix ends with bucket bprev
+      double m2, k2;
+      long long c2, kc2;
+      gathered_bucket_stats(sm, m, bprev, 0u, m2, c2, k2, kc2, kmin);
+    }
+    best = Cut{kmin, before_mu + kcnt, P.a_mu + kmass};
+    have = true;
+  }
+  if (p_on) {
+    const double target = (double)p * P.z;
+    // the crossing bucket, from the exact masses of the gathered window
+    double wm[3];
+    long long wc[3];
+    window_stats(sm, m, lo, hi, wm, wc);
+    double before = P.a_p;
+    long long cbefore = before_win;
+    int c = -1;
+    for (int w = lo; w <= hi; ++w) {
+      if (before < target && target <= before + wm[w - lo]) {
+        c = w;
+        break;
+      }
+      before += wm[w - lo];
+      cbefore += wc[w - lo];
+    }
+    if (c < 0) return false;  // the crossing lies outside the window
+    const int n = compact_gathered(sm, m, c, c);
+    sort_and_scan(sm, 0, n, m);
+    const int jp = first_mass_hit(sm, 0, n, before, 0.0, kMassGE, target);
+    const Cut cp{sm.cand[jp], cbefore + jp + 1, before + sm.cq[jp]};
+    if (have)
+      take_earlier(best, cp);
+    else
+      best = cp;
+  }
+  __syncthreads();
+  return true;
 }
 
 template <bool VEC>
@@ -624,6 +1133,7 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
   RSmem& sm = *reinterpret_cast<RSmem*>(smem_raw);
   const int V = a.V;
   for (int i = threadIdx.x; i < NB; i += RT) sm.tab[i] = exp(-(double)i * (1.0 / 128.0));
+  if (threadIdx.x == 0) sm.bd[3] = exp(-1.0 / 256.0);  // mid-bucket weight factor
   __syncthreads();
 
   for (int r = blockIdx.x; r < a.rows; r += gridDim.x) {
@@ -658,19 +1168,12 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
     const float m = block_max_f(lm, sm);
     const double md = (double)m;
 
-    double Z;
-    unsigned long long Klast;
-    build_hist0<VEC>(sm, x, V, m, &Z, &Klast);
-    bool hist_valid = true;
-    Cut best{Klast, (long long)V, Z};
-
     const int k = a.top_k[r];
     const float p = a.top_p[r];
     const float mu = a.min_p[r];
     const bool k_on = k >= 1 && k < V;
     const bool p_on = p < 1.0f;
     const bool mu_on = mu > 0.0f;
-    bool ok = true;
 
     uint32_t kt = 0;
     if (mu_on) {
@@ -680,95 +1183,10 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
       __syncthreads();
     }
 
-    bool done = false;
-    double Zk = Z;
-    if (k_on) {
-      int bk;
-      long long ce;
-      double me;
-      pick_bucket(sm, kCount, (long long)k, 0.0, 0, 0.0, bk, ce, me);
-      const long long incl = ce + sm.cnt[bk];
-      __syncthreads();
-      if (incl <= CAP) {
-        // small k: the whole prefix of buckets [0, bk] fits, and every cut
-        // that can be earlier than the top-k cut lies inside it
-        const int n = gather_prefix<VEC>(sm, x, V, m, bk);
-        sort_and_scan(sm, n, m);
-        const int jk = min(k, n) - 1;
-        Cut ck{sm.cand[jk], (long long)jk + 1, sm.cq[jk]};
-        Zk = ck.mass;
-        take_earlier(best, ck);
-        if (p_on) {
-          const int jp = first_mass_hit(sm, 0, jk + 1, 0.0, 0.0, kMassGE, (double)p * Zk);
-          take_earlier(best, Cut{sm.cand[jp], (long long)jp + 1, sm.cq[jp]});
-        }
-        if (mu_on) {
-          // kept candidates form a prefix; count them
-          int mine = 0;
-          for (int j = threadIdx.x; j < n; j += RT) mine += (uint32_t)(sm.cand[j] >> 32) >= kt ? 1 : 0;
-          const int nk = (int)block_sum_l(mine, sm);
-          if (nk >= 1 && nk < n) take_earlier(best, Cut{sm.cand[nk - 1], (long long)nk, sm.cq[nk - 1]});
-        }
-        __syncthreads();
-        done = true;
-      } else {
-        Cut ck;
-        ok = locate<VEC>(sm, x, V, m, hist_valid, kCount, (long long)k, 0.0, ck);
-        Zk = ck.mass;
-        take_earlier(best, ck);
-      }
-    }
-
-    if (ok && !done && (p_on || mu_on)) {
-      if (!hist_valid) {
-        build_hist0<VEC>(sm, x, V, m, nullptr, nullptr);
-        hist_valid = true;
-      }
-      const double target = (double)p * Zk;
-      int bp = -1, bm = -1;
-      long long cp_excl = 0, cm_excl = 0;
-      double mp_excl = 0.0, mm_excl = 0.0;
-      if (p_on) pick_bucket(sm, kMassGE, 0, target, 0, 0.0, bp, cp_excl, mp_excl);
-      if (mu_on) {
-        bm = bin0(key32_value(kt), m);
-        bucket_prefix(sm, bm, cm_excl, mm_excl);
-      }
-      const int np_ = bp >= 0 ? sm.cnt[bp] : 0;
-      const int nm_ = (bm >= 0 && bm != bp) ? sm.cnt[bm] : 0;
-      __syncthreads();
-      if (np_ + nm_ <= CAP) {
-        // one pass gathers both boundary buckets and the last min-p element
-        unsigned long long K_mu = 0ull;
-        const int n = gather_two<VEC>(sm, x, V, m, bp, bm, mu_on, kt, &K_mu);
-        sort_and_scan(sm, n, m);
-        // sorted candidates: the earlier bucket's run first
-        if (p_on) {
-          const int lo = (bm >= 0 && bm < bp) ? nm_ : 0;
-          const double before = lo > 0 ? sm.cq[lo - 1] : 0.0;
-          const int jp = first_mass_hit(sm, lo, lo + np_, mp_excl, before, kMassGE, target);
-          take_earlier(best, Cut{sm.cand[jp], cp_excl + (jp - lo) + 1, mp_excl + (sm.cq[jp] - before)});
-        }
-        if (mu_on) {
-          const int lo = (bp >= 0 && bp < bm) ? np_ : 0;
-          const int cntb = sm.cnt[bm];
-          int mine = 0;
-          for (int j = lo + (int)threadIdx.x; j < lo + cntb; j += RT)
-            mine += (uint32_t)(sm.cand[j] >> 32) >= kt ? 1 : 0;
-          const int nk = (int)block_sum_l(mine, sm);
-          const double before = lo > 0 ? sm.cq[lo - 1] : 0.0;
-          const double mass = mm_excl + (nk > 0 ? sm.cq[lo + nk - 1] - before : 0.0);
-          take_earlier(best, Cut{K_mu, cm_excl + nk, mass});
-        }
-        __syncthreads();
-      } else {
-        if (p_on) {
-          Cut cp;
-          ok = locate<VEC>(sm, x, V, m, hist_valid, kMassGE, 0, target, cp);
-          take_earlier(best, cp);
-        }
-        if (ok && mu_on) take_earlier(best, min_p_cut_pass<VEC>(sm, x, V, m, kt));
-      }
-    }
+    Cut best;
+    bool hist_valid = false;
+    bool ok = resolve_row_fast<VEC>(sm, x, V, m, k, p, mu, kt, best);
+    if (!ok) ok = resolve_row_exact<VEC>(sm, x, V, m, k, p, mu, kt, hist_valid, best);
 
     if (!ok) {
       if (threadIdx.x == 0) {
