@@ -150,6 +150,28 @@ sts_status sts_filter_logits(const sts_shape* shape, const float* scaled_logits,
                              int32_t* cut_id, uint8_t* mask, void* ws, size_t ws_bytes,
                              sts_stream_t stream);
 
+/* sts_filter_logits for callers that cannot allocate device memory: code
+ * running under a fixed device-memory reservation (where cudaMalloc may fail,
+ * or implicitly synchronise the device in the middle of a step), or code
+ * called from inside an allocator or framework callback that must not
+ * re-enter the allocator. The pages have no counterpart: this entry point
+ * exists for such callers, not for the method.
+ * Same inputs, outputs and results as sts_filter_logits, minus the workspace:
+ * the scratch (a 256-byte status header plus one int32 per row) is a
+ * file-scope device array of 262,400 bytes that every GPU loading the library
+ * holds until process exit. T must be <= 65,536 (else STS_ERR_SHAPE).
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the array, which keeps the last call's contents (the header
+ * is cleared at the start of each call): calls that overlap on the GPU -- on
+ * different streams, or from different host threads -- race. Row-value
+ * errors show per row (support_size 0, cut_id -1, cut_logit NaN); there is
+ * no status word to read back. Allocates nothing. */
+sts_status sts_filter_logits_noalloc(const sts_shape* shape, const float* scaled_logits,
+                                     const sts_rows* rows, int32_t* support_size,
+                                     float* cut_logit, int32_t* cut_id, uint8_t* mask,
+                                     sts_stream_t stream);
+
 /* Test hook: the forward's first pass alone, S[t, v] = (H . W^T)[t, v] /
  * temperature[t] for t in [t0, t0 + rows), v in [v0, v0 + cols), written to
  * S_out[(t - t0) * ld + (v - v0)] (fp32). t0 must be a multiple of 128 and v0

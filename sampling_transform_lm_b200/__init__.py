@@ -37,6 +37,7 @@ __all__ = [
     "sts_launch_count",
     "sts_timing_enable",
     "sts_timing_read",
+    "sts_filter_logits_noalloc",
     "KERNEL_KINDS",
     "ROW_TARGET_IN_SUPPORT",
     "ROW_INVALID",
@@ -72,6 +73,7 @@ EXPORTED_SYMBOLS = (
     "sts_launch_count",
     "sts_timing_enable",
     "sts_timing_read",
+    "sts_filter_logits_noalloc",
 )
 
 
@@ -144,6 +146,9 @@ def load():
     lib.sts_timing_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(ctypes.c_int64)]
     lib.sts_timing_read.restype = ctypes.c_int
+    lib.sts_filter_logits_noalloc.argtypes = [ctypes.POINTER(_Shape), P, ctypes.POINTER(_Rows), P, P,
+                                              P, P, P]
+    lib.sts_filter_logits_noalloc.restype = ctypes.c_int
     lib.sts_abi_version.argtypes = []
     lib.sts_abi_version.restype = ctypes.c_int
     _lib = lib
@@ -336,6 +341,27 @@ def sts_filter_logits(S, top_k, top_p, min_p, *, want_mask=False, ws=None, strea
     if check:
         sts_get_status(ws, stream, raise_on_error=True)
     return {"size": size, "cut_logit": cut_logit, "cut_id": cut_id, "mask": mask}
+
+
+def sts_filter_logits_noalloc(S, top_k, top_p, min_p, *, support_size, cut_logit, cut_id,
+                              mask=None, stream=None):
+    """sts_filter_logits without a workspace, for callers that cannot allocate
+    device memory: every output is caller-provided and the C entry point
+    allocates nothing (its scratch is a fixed device array, T <= 65,536)."""
+    lib = load()
+    _need(S, torch.float32, "S")
+    T, V = S.shape
+    for name, t, dt in (("top_k", top_k, torch.int32), ("top_p", top_p, torch.float32),
+                        ("min_p", min_p, torch.float32), ("support_size", support_size, torch.int32),
+                        ("cut_logit", cut_logit, torch.float32), ("cut_id", cut_id, torch.int32)):
+        _need(t, dt, name, (T,))
+    if mask is not None:
+        _need(mask, torch.uint8, "mask", (T, V))
+    rows = _Rows(T, None, None, _ptr(top_k), _ptr(top_p), _ptr(min_p))
+    sh = _shape(T, 8, V)
+    _check(lib.sts_filter_logits_noalloc(ctypes.byref(sh), _ptr(S), ctypes.byref(rows),
+                                         _ptr(support_size), _ptr(cut_logit), _ptr(cut_id),
+                                         _ptr(mask), _stream(stream)), "sts_filter_logits_noalloc")
 
 
 def sts_scaled_logits(H, W, temperature, t0=0, rows=None, v0=0, cols=None, *, out=None,
