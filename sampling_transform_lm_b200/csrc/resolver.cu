@@ -763,7 +763,11 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
   double z[2] = {0.0, 0.0}, ap[2] = {0.0, 0.0}, amu[2] = {0.0, 0.0};
   unsigned long long kl = ~0ull;
 
-  auto batch = [&](const float (&sv)[E], int i0, int nvalid) {
+  // Element e < 4 of a batch is token a0 + e (valid when e < na), element
+  // e >= 4 is token b0 + e - 4 (valid when e - 4 < nb).
+  auto batch = [&](const float (&sv)[E], int a0, int na, int b0, int nb) {
+    auto idx = [&](int e) { return e < 4 ? a0 + e : b0 + (e - 4); };
+    auto valid = [&](int e) { return e < 4 ? e < na : e - 4 < nb; };
     int bb[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) bb[e] = bin0(sv[e], m);
@@ -787,7 +791,7 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
         if (bb[e] >= NB - 1) qq[e] = exp((double)sv[e] - md);
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const double q = e < nvalid ? qq[e] : 0.0;
+        const double q = valid(e) ? qq[e] : 0.0;
         z[e & 1] += q;
         ap[e & 1] += bb[e] < w_lo ? q : 0.0;
         amu[e & 1] += bb[e] < b_mu ? q : 0.0;
@@ -795,68 +799,60 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
     } else {
 #pragma unroll
       for (int e = 0; e < E; ++e)
-        if (e < nvalid && bb[e] < b_mu) amu[e & 1] += qmass_b(sm.tab, sv[e], md, bb[e]);
+        if (valid(e) && bb[e] < b_mu) amu[e & 1] += qmass_b(sm.tab, sv[e], md, bb[e]);
     }
     if (need_last) {
 #pragma unroll
       for (int e = 0; e < E; ++e)
-        if (e < nvalid) {
-          const unsigned long long K = ckey(sv[e], i0 + e);
+        if (valid(e)) {
+          const unsigned long long K = ckey(sv[e], idx(e));
           kl = K < kl ? K : kl;
         }
     }
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const int b = bb[e];
-      const bool g = e < nvalid && ((b >= g_lo && b <= g_hi) || (b >= g2_lo && b <= g2_hi));
+      const bool g = valid(e) && ((b >= g_lo && b <= g_hi) || (b >= g2_lo && b <= g2_hi));
       const unsigned mask = __ballot_sync(0xffffffffu, g);
       if (mask) {
         const int slot = wfill + __popc(mask & lt);
-        if (g && slot < WCAP) wbuf[slot] = ckey(sv[e], i0 + e);
+        if (g && slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
         wfill += __popc(mask);
       }
     }
   };
 
+  const int tid = (int)threadIdx.x;
+  int tail0 = 0;  // first token handled one per thread
   if (VEC) {
+    // Fully coalesced: in each sweep thread t reads float4s base + u * RT + t
+    // (u = 0..3), so every warp load covers 512 contiguous bytes; a batch
+    // pairs two of those float4s.
     const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
-    const int V8 = V / E;  // batches of 8 consecutive elements (two float4)
-    for (int base = 0; base < V8; base += RT * 2) {
-      float4 va[2], vb[2];
+    const int V4 = V >> 2;
+    for (int base = 0; base < V4; base += RT * 4) {
+      float4 v[4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int i = base + u * RT + (int)threadIdx.x;
-        if (i < V8) {
-          va[u] = ld_stream4(x4 + 2 * i);
-          vb[u] = ld_stream4(x4 + 2 * i + 1);
-        } else {
-          va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + u * RT + tid;
+        v[u] = i < V4 ? ld_stream4(x4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll 1
-      for (int u = 0; u < 2; ++u) {
-        const int i = base + u * RT + (int)threadIdx.x;
-        const float sv[E] = {va[u].x, va[u].y, va[u].z, va[u].w, vb[u].x, vb[u].y, vb[u].z, vb[u].w};
-        batch(sv, E * i, i < V8 ? E : 0);
+      for (int h = 0; h < 2; ++h) {
+        const int ia = base + 2 * h * RT + tid, ib = ia + RT;
+        const float4 a4 = h ? v[2] : v[0], b4 = h ? v[3] : v[1];
+        const float sv[E] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+        batch(sv, 4 * ia, ia < V4 ? 4 : 0, 4 * ib, ib < V4 ? 4 : 0);
       }
     }
-    for (int i0 = E * V8; i0 < V; i0 += RT) {
-      const int i = i0 + (int)threadIdx.x;
-      float sv[E];
-      const float v = i < V ? ld_stream(x + i) : 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) sv[e] = v;
-      batch(sv, i, i < V ? 1 : 0);
-    }
-  } else {
-    for (int i0 = 0; i0 < V; i0 += RT) {
-      const int i = i0 + (int)threadIdx.x;
-      float sv[E];
-      const float v = i < V ? ld_stream(x + i) : 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) sv[e] = v;
-      batch(sv, i, i < V ? 1 : 0);
-    }
+    tail0 = 4 * V4;
+  }
+  for (int i0 = tail0; i0 < V; i0 += RT) {
+    const int i = i0 + tid;
+    const bool in = i < V;
+    const float t = in ? ld_stream(x + i) : 0.f;
+    const float sv[E] = {t, t, t, t, t, t, t, t};
+    batch(sv, i, in ? 1 : 0, i, 0);
   }
   if (lane == 0) sm.wcount[warp] = wfill;
   double sums[3] = {z[0] + z[1], ap[0] + ap[1], amu[0] + amu[1]};
