@@ -19,15 +19,33 @@
 //   support    the shortest of the three prefixes; its size, mass Z_S and
 //              last element (the cut) give LSE_S = m + log Z_S
 //
-// Work per row: one streaming pass builds a 4096-bucket histogram (count and
-// float64 mass) with buckets uniform in (m - s) -- floor((m - s) * 128),
-// clamped to 4095 -- which is monotone in s, so every bucket is a contiguous
-// run of the order. The buckets that hold a cut are then gathered in one more
-// pass (from L2), sorted by composite key and scanned, which places each cut
-// exactly. A bucket too large for the 4096-entry candidate buffer is split
-// again on its composite keys (12 bits per level) until it fits; the keys are
-// distinct, so this ends after at most six levels. The row max comes from the
-// projection's epilogue (one partial max per 256-column tile) when available.
+// Work per row (one 512-thread CTA per SM, persistent over rows; a row's
+// metadata and the projection epilogue's per-tile maxima, which give the
+// unfiltered max m, are loaded one row ahead):
+//
+//   count pass   a 4096-bucket count histogram with buckets uniform in m - s
+//                (floor((m - s) * 128), clamped to 4095). The bucket index is
+//                monotone in s, so every bucket is a contiguous run of the
+//                order.
+//   planning     from the counts alone: the top-k cut's bucket; the top-p
+//                crossing's bucket estimated with mid-bucket weights, widened
+//                to a 3-bucket window; the min-p threshold's bucket and the
+//                non-empty bucket before it.
+//   exact pass   (from L2) float64 masses of every element, summed in
+//                registers (the total, the mass before the window, the mass
+//                before the min-p bucket), and the elements of the planned
+//                buckets gathered into per-warp slices of a candidate buffer.
+//   finish       exact masses of the window buckets place the crossing in one
+//                bucket; its elements are sorted by composite key (a bitonic
+//                network held mostly in registers and warp shuffles) and
+//                scanned, which places each cut exactly.
+//
+// When the plan cannot be proven to hold a cut (a crossing outside the
+// window, too many candidates, large top-k) the row falls back to the exact
+// search: a float64 mass histogram, then the candidate buckets gathered from
+// the row, refining a bucket too large for the 4096-entry sort on its
+// composite keys (12 bits per level) until it fits; the keys are distinct, so
+// this ends after at most six levels.
 //
 // Masses use a table-driven float64 exponential (P. T. P. Tang, "Table-driven
 // implementation of the exponential function in IEEE floating-point
@@ -49,15 +67,31 @@ constexpr int RT = 512;             // threads per resolver CTA
 constexpr int NWARP = RT / 32;
 constexpr int NB = 4096;            // histogram buckets per level
 constexpr int CAP = 8192;           // candidate buffer (composite keys)
+constexpr int SCAP = 4096;          // candidates sorted and scanned at once
 constexpr float BIN_SCALE = 128.f;  // level-0 buckets per logit unit
 constexpr int MAX_LEVELS = 8;
 constexpr int UNROLL = 4;           // float4 loads in flight per thread
 
+// exp(-b / 128) for every bucket b.
+struct ExpTab {
+  double v[NB];
+};
+
+__device__ __forceinline__ double tab_at(const ExpTab& t, int b) { return t.v[b]; }
+
+__device__ void init_exp_tab(ExpTab& t, int tid, int nthreads) {
+  for (int i = tid; i < NB; i += nthreads) t.v[i] = exp(-(double)i * (1.0 / 128.0));
+}
+
+// The bucket masses (planning and the exact histogram) and the candidates'
+// mass scan are never live at once and share storage.
 struct RSmem {
-  double mass[NB];
-  double tab[NB];  // exp(-b / 128)
+  union {
+    double mass[NB];
+    double cq[SCAP];  // inclusive mass scan of at most SCAP sorted candidates
+  };
   unsigned long long cand[CAP];
-  double cq[CAP / 2];  // inclusive mass scan of at most CAP / 2 sorted candidates
+  ExpTab tab;
   int cnt[NB];
   double red_d[NWARP];
   double red_m[NWARP * 8 + 8];
@@ -90,6 +124,7 @@ __device__ __forceinline__ unsigned long long ckey(float s, int id) {
 
 __device__ __forceinline__ float ckey_value(unsigned long long K) { return key32_value((uint32_t)(K >> 32)); }
 
+
 __device__ __forceinline__ int ckey_id(unsigned long long K) {
   return (int)(0xFFFFFFFFu - (uint32_t)(K & 0xFFFFFFFFull));
 }
@@ -100,10 +135,14 @@ __device__ __forceinline__ int bin0(float s, float m) {
   return b < 0 ? 0 : b;
 }
 
+// exp(x) for the far tail (x < -32), kept out of line so the loops that
+// stream a row do not carry its registers.
+__device__ __noinline__ double far_mass(double x) { return exp(x); }
+
 // exp((double)s - (double)m) for an element in level-0 bucket b.
-__device__ __forceinline__ double qmass_b(const double* tab, float s, double md, int b) {
+__device__ __forceinline__ double qmass_b(const ExpTab& tab, float s, double md, int b) {
   const double x = (double)s - md;
-  if (b >= NB - 1) return exp(x);
+  if (b >= NB - 1) return far_mass(x);
   const double r = x + (double)b * (1.0 / 128.0);
   double p = 1.0 / 720.0;
   p = fma(p, r, 1.0 / 120.0);
@@ -112,7 +151,7 @@ __device__ __forceinline__ double qmass_b(const double* tab, float s, double md,
   p = fma(p, r, 0.5);
   p = fma(p, r, 1.0);
   p = fma(p, r, 1.0);
-  return tab[b] * p;
+  return tab_at(tab, b) * p;
 }
 
 __device__ __forceinline__ double qmass(const RSmem& sm, float s, float m) {
@@ -311,6 +350,50 @@ __device__ T block_exscan(T v, T* warp_tot, T& total) {
   return before_warp + x - v;
 }
 
+// Exclusive scans of a count and a mass over threads in thread order, in one
+// exchange.
+__device__ void block_exscan2(long long a, double b, long long& pa, double& pb, long long& ta,
+                              double& tb, RSmem& sm) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  long long xa = a;
+  double xb = b;
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long ya = __shfl_up_sync(0xffffffffu, xa, o);
+    const double yb = __shfl_up_sync(0xffffffffu, xb, o);
+    if (l >= o) {
+      xa += ya;
+      xb += yb;
+    }
+  }
+  if (l == 31) {
+    sm.red_l[w] = xa;
+    sm.red_d[w] = xb;
+  }
+  __syncthreads();
+  if (w == 0) {
+    long long s = l < NWARP ? sm.red_l[l] : 0;
+    double d = l < NWARP ? sm.red_d[l] : 0.0;
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long ys = __shfl_up_sync(0xffffffffu, s, o);
+      const double yd = __shfl_up_sync(0xffffffffu, d, o);
+      if (l >= o) {
+        s += ys;
+        d += yd;
+      }
+    }
+    if (l < NWARP) {
+      sm.red_l[l] = s;  // inclusive warp prefixes
+      sm.red_d[l] = d;
+    }
+  }
+  __syncthreads();
+  pa = (w > 0 ? sm.red_l[w - 1] : 0) + xa - a;
+  pb = (w > 0 ? sm.red_d[w - 1] : 0.0) + xb - b;
+  ta = sm.red_l[NWARP - 1];
+  tb = sm.red_d[NWARP - 1];
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------- selection
 
 enum Crit : int { kCount = 0, kMassGE = 1, kMassGT = 2 };
@@ -410,65 +493,105 @@ __device__ __noinline__ void build_hist0(RSmem& sm, const float* __restrict__ x,
   if (Kmin) *Kmin = block_ext_u<false>(kl, sm);
 }
 
-// Sort sm.cand[0..n) descending (composite keys are distinct) and write the
-// inclusive float64 prefix of the masses to sm.cq (thread order, deterministic).
-// Sorts the n (<= CAP / 2) candidates of sm.cand[a0, a0 + n) into
-// sm.cand[0, n) and writes their inclusive mass scan to sm.cq[0, n) (the rest
-// of the candidate buffer is scratch afterwards).
-__device__ __noinline__ void sort_and_scan(RSmem& sm, int a0, int n, float m) {
-  constexpr int PER = (CAP / 2) / RT;
-  n = min(n, CAP / 2);
-  if (a0 != 0) {
-    unsigned long long t[PER];
+// Bitonic sort of sm.cand[0, n) into descending order (composite keys are
+// distinct), then the inclusive float64 scan of their masses into sm.cq[0, n)
+// (thread order, deterministic). The first NW warps sort a padded run of
+// N2 = 32 * NW * E keys: element i = t * E + e lives in register v[e] of
+// thread t, so compare-exchange partners closer than E are in one thread,
+// partners closer than 32 E are a warp shuffle away, and only the wider stages
+// (log2(NW) (log2(NW) + 1) / 2 of them) go through shared memory, one barrier
+// each, alternating between the two halves of sm.cand. Padding keys are 0 and
+// sort last.
+template <int E, int NW>
+__device__ void sort_scan_regs(RSmem& sm, int n, float m) {
+  constexpr int N2 = 32 * NW * E;
+  static_assert(NW <= NWARP && 2 * N2 <= CAP, "two shared-stage buffers fit the candidate buffer");
+  const int t = (int)threadIdx.x;
+  const bool part = t < 32 * NW;  // whole warps: shuffles stay within a warp
+  unsigned long long v[E];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int j = (int)threadIdx.x * PER + i;
-      t[i] = j < n ? sm.cand[a0 + j] : 0ull;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int j = (int)threadIdx.x * PER + i;
-      if (j < n) sm.cand[j] = t[i];
-    }
-    __syncthreads();
+  for (int e = 0; e < E; ++e) {
+    const int i = t * E + e;
+    v[e] = (part && i < n) ? sm.cand[i] : 0ull;
   }
-  unsigned long long* c = sm.cand;
-  int n2 = 2;
-  while (n2 < n) n2 <<= 1;
-  for (int i = n + (int)threadIdx.x; i < n2; i += RT) c[i] = 0ull;  // sorts last
-  __syncthreads();
-  for (int k = 2; k <= n2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += RT) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long x0 = c[i], x1 = c[ixj];
-          const bool desc = (i & k) == 0;
-          if (desc ? (x0 < x1) : (x0 > x1)) {
-            c[i] = x1;
-            c[ixj] = x0;
-          }
+  int buf = 0;
+  for (int k = 2; k <= N2; k <<= 1) {
+    int j = k >> 1;
+    for (; j >= 32 * E; j >>= 1) {  // across warps: through shared memory
+      unsigned long long* c = sm.cand + buf * N2;
+      if (part)
+#pragma unroll
+        for (int e = 0; e < E; ++e) c[t * E + e] = v[e];
+      __syncthreads();
+      if (part)
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = t * E + e;
+          const unsigned long long o = c[i ^ j];
+          const bool keep_hi = ((i & j) == 0) == ((i & k) == 0);
+          v[e] = keep_hi ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+        }
+      buf ^= 1;
+    }
+    for (; j >= E; j >>= 1) {  // across lanes: warp shuffles
+      const int lj = j / E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int i = t * E + e;
+        const unsigned long long o = __shfl_xor_sync(0xffffffffu, v[e], lj);
+        const bool keep_hi = ((i & j) == 0) == ((i & k) == 0);
+        v[e] = keep_hi ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+      }
+    }
+#pragma unroll
+    for (int jj = E / 2; jj > 0; jj >>= 1) {  // within the thread
+      if (jj >= k) continue;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int q = e ^ jj;
+        if (q > e) {
+          const bool desc = ((t * E + e) & k) == 0;
+          const unsigned long long x0 = v[e], x1 = v[q];
+          const unsigned long long hi = x0 > x1 ? x0 : x1, lo = x0 > x1 ? x1 : x0;
+          v[e] = desc ? hi : lo;
+          v[q] = desc ? lo : hi;
         }
       }
-      __syncthreads();
     }
   }
-  const int base = threadIdx.x * PER;
-  double loc[PER];
+  double loc[E];
   double run = 0.0;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int j = base + i;
-    const double qv = j < n ? qmass(sm, ckey_value(c[j]), m) : 0.0;
-    run += qv;
-    loc[i] = run;
+  for (int e = 0; e < E; ++e) {
+    const int i = t * E + e;
+    run += (part && i < n) ? qmass(sm, ckey_value(v[e]), m) : 0.0;
+    loc[e] = run;
   }
   double tot;
-  const double off = block_exscan<double>(run, sm.red_d, tot);
+  const double off = block_exscan<double>(run, sm.red_d, tot);  // its barriers end the shared stages
+  if (part)
 #pragma unroll
-  for (int i = 0; i < PER; ++i) sm.cq[base + i] = off + loc[i];
+    for (int e = 0; e < E; ++e) {
+      const int i = t * E + e;
+      sm.cand[i] = v[e];
+      sm.cq[i] = off + loc[e];
+    }
   __syncthreads();
+}
+
+// Sorts sm.cand[0, n) (n <= SCAP) and scans the masses into sm.cq[0, n).
+__device__ __noinline__ void sort_and_scan(RSmem& sm, int n, float m) {
+  n = min(n, SCAP);
+  if (n <= 64)
+    sort_scan_regs<2, 1>(sm, n, m);  // one warp, no shared stage
+  else if (n <= 256)
+    sort_scan_regs<2, 4>(sm, n, m);
+  else if (n <= 1024)
+    sort_scan_regs<2, NWARP>(sm, n, m);
+  else if (n <= 2048)
+    sort_scan_regs<4, NWARP>(sm, n, m);
+  else
+    sort_scan_regs<8, NWARP>(sm, n, m);
 }
 
 // First j in [lo, hi) with C(j) = base_mass + (cq[j] - cq_before) meeting a
@@ -520,7 +643,7 @@ __device__ __noinline__ bool locate(RSmem& sm, const float* __restrict__ x, int 
   bool refined = false;
   __syncthreads();
 
-  for (int level = 0; set_cnt > CAP / 2; ++level) {
+  for (int level = 0; set_cnt > SCAP; ++level) {
     if (level >= MAX_LEVELS) return false;
     unsigned long long kmin = ~0ull, kmax = 0ull;
     for_each<VEC>(x, V, [&](float s, int i) {
@@ -578,7 +701,8 @@ __device__ __noinline__ bool locate(RSmem& sm, const float* __restrict__ x, int 
   });
   __syncthreads();
   const int n = min(sm.ncand, CAP);
-  sort_and_scan(sm, 0, n, m);
+  sort_and_scan(sm, n, m);
+  hist_valid = false;  // the scan overwrote the bucket masses
   int jstar;
   if (crit == kCount)
     jstar = (int)(need - above_cnt - 1);
@@ -740,6 +864,14 @@ struct Plan2 {
 };
 
 constexpr int WCAP = CAP / NWARP;  // private gather slots per warp
+// Readers of the slices take slot i * RT + tid (i < CAP / RT), which is
+// position (i % SLR) * RT + tid of slice i / SLR: a warp reads 32 consecutive
+// keys (no bank conflicts).
+constexpr int SLR = WCAP / RT;  // reader steps per slice
+static_assert(WCAP % RT == 0, "a slice is a whole number of reader steps");
+__device__ __forceinline__ bool slot_live(const RSmem& sm, int i) {
+  return (i % SLR) * RT + (int)threadIdx.x < sm.wcount[i / SLR];
+}
 
 // One pass over the row: exact float64 masses accumulated in registers, and
 // the elements of up to two bucket ranges gathered into per-warp slices of
@@ -754,6 +886,8 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
   constexpr int E = 8;
   const double md = (double)m;
   const bool need_last = pl.need_last != 0;
+  // bucket ranges as (start, span) for one unsigned compare each; an empty
+  // range starts past the last bucket
   const int g_lo = pl.g_lo, g_hi = pl.g_hi, g2_lo = pl.g2_lo, g2_hi = pl.g2_hi;
   const int w_lo = pl.w_lo, b_mu = pl.b_mu;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -764,15 +898,20 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
   unsigned long long kl = ~0ull;
 
   // Element e < 4 of a batch is token a0 + e (valid when e < na), element
-  // e >= 4 is token b0 + e - 4 (valid when e - 4 < nb).
+  // e >= 4 is token b0 + e - 4 (valid when e - 4 < nb). The body has no
+  // per-element branches: masses are computed for all E elements and
+  // selected, the far tail (bucket NB - 1) takes one warp vote per batch, and
+  // each gather store is predicated on its ballot rather than branched over.
+  const bool need_mass = NEED_Z || b_mu >= 0;
   auto batch = [&](const float (&sv)[E], int a0, int na, int b0, int nb) {
     auto idx = [&](int e) { return e < 4 ? a0 + e : b0 + (e - 4); };
-    auto valid = [&](int e) { return e < 4 ? e < na : e - 4 < nb; };
+    auto ok = [&](int e) { return e < 4 ? e < na : e - 4 < nb; };
     int bb[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) bb[e] = bin0(sv[e], m);
-    if (NEED_Z) {
+    if (need_mass) {
       double qq[E];
+      bool far = false;
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         const double xx = (double)sv[e] - md;
@@ -784,41 +923,39 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
         p = fma(p, r, 0.5);
         p = fma(p, r, 1.0);
         p = fma(p, r, 1.0);
-        qq[e] = sm.tab[bb[e]] * p;
+        qq[e] = tab_at(sm.tab, bb[e]) * p;
+        far |= bb[e] >= NB - 1;
       }
+      if (__any_sync(0xffffffffu, far)) {
 #pragma unroll
-      for (int e = 0; e < E; ++e)
-        if (bb[e] >= NB - 1) qq[e] = exp((double)sv[e] - md);
+        for (int e = 0; e < E; ++e)
+          if (bb[e] >= NB - 1) qq[e] = far_mass((double)sv[e] - md);
+      }
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const double q = valid(e) ? qq[e] : 0.0;
-        z[e & 1] += q;
-        ap[e & 1] += bb[e] < w_lo ? q : 0.0;
+        const double q = ok(e) ? qq[e] : 0.0;
+        if (NEED_Z) {
+          z[e & 1] += q;
+          ap[e & 1] += bb[e] < w_lo ? q : 0.0;
+        }
         amu[e & 1] += bb[e] < b_mu ? q : 0.0;
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e)
-        if (valid(e) && bb[e] < b_mu) amu[e & 1] += qmass_b(sm.tab, sv[e], md, bb[e]);
     }
     if (need_last) {
 #pragma unroll
-      for (int e = 0; e < E; ++e)
-        if (valid(e)) {
-          const unsigned long long K = ckey(sv[e], idx(e));
-          kl = K < kl ? K : kl;
-        }
+      for (int e = 0; e < E; ++e) {
+        const unsigned long long K = ok(e) ? ckey(sv[e], idx(e)) : ~0ull;
+        kl = K < kl ? K : kl;
+      }
     }
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const int b = bb[e];
-      const bool g = valid(e) && ((b >= g_lo && b <= g_hi) || (b >= g2_lo && b <= g2_hi));
-      const unsigned mask = __ballot_sync(0xffffffffu, g);
-      if (mask) {
-        const int slot = wfill + __popc(mask & lt);
-        if (g && slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
-        wfill += __popc(mask);
-      }
+      const bool g = ok(e) && ((b >= g_lo && b <= g_hi) || (b >= g2_lo && b <= g2_hi));
+      const unsigned mk = __ballot_sync(0xffffffffu, g);
+      const int slot = wfill + __popc(mk & lt);
+      if (g && slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
+      wfill += __popc(mk);
     }
   };
 
@@ -878,31 +1015,30 @@ __device__ void pass2(RSmem& sm, const float* __restrict__ x, int V, float m, bo
 
 // Move the gathered candidates whose bucket lies in [lo, hi] from the per-warp
 // slices to sm.cand[0, n) (block scan, order irrelevant: they are sorted
-// next). Returns n.
+// next). At most SCAP are kept. Returns n.
 __device__ __noinline__ int compact_gathered(RSmem& sm, float m, int lo, int hi) {
-  constexpr int PER = CAP / RT;  // slots per thread (inside one warp slice)
+  constexpr int PER = CAP / RT;
   unsigned long long t[PER];
   int mine = 0;
-  const int base = (int)threadIdx.x * PER;
-  const int wcnt = sm.wcount[base / WCAP];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
-    const int slot = base + i;
-    const bool ok = (slot % WCAP) < wcnt;
-    const unsigned long long K = ok ? sm.cand[slot] : 0ull;
-    const int b = ok ? bin0(ckey_value(K), m) : -1;
-    t[i] = (ok && b >= lo && b <= hi) ? K : 0ull;
+    const bool live = slot_live(sm, i);
+    const unsigned long long K = live ? sm.cand[i * RT + threadIdx.x] : 0ull;
+    const int b = bin0(ckey_value(K), m);
+    t[i] = (live && b >= lo && b <= hi) ? K : 0ull;
     mine += t[i] != 0ull ? 1 : 0;
   }
   long long tot;
-  const int off = (int)block_exscan<long long>((long long)mine, sm.red_l, tot);
-  // t[] holds this thread's share; the buffer is rewritten from the front
-  int o = off;
+  int o = (int)block_exscan<long long>((long long)mine, sm.red_l, tot);
+  // every slot is in registers now: the buffer is rewritten from the front
 #pragma unroll
   for (int i = 0; i < PER; ++i)
-    if (t[i] != 0ull) sm.cand[o++] = t[i];
+    if (t[i] != 0ull) {
+      if (o < SCAP) sm.cand[o] = t[i];
+      ++o;
+    }
   __syncthreads();
-  return (int)tot;
+  return (int)min(tot, (long long)SCAP);
 }
 
 // Exact mass and count of the gathered candidates in bucket b, and (for
@@ -911,30 +1047,29 @@ __device__ __noinline__ void gathered_bucket_stats(RSmem& sm, float m, int b, ui
                                                    double& mass, long long& cnt, double& kept_mass,
                                                    long long& kept_cnt, unsigned long long& k_min) {
   constexpr int PER = CAP / RT;
-  const int base = (int)threadIdx.x * PER;
-  const int wcnt = sm.wcount[base / WCAP];
   double ms = 0.0, km = 0.0;
   long long c = 0, kc = 0;
   unsigned long long kmn = ~0ull;
+#pragma unroll 4
   for (int i = 0; i < PER; ++i) {
-    const int slot = base + i;
-    if ((slot % WCAP) >= wcnt) continue;
-    const unsigned long long K = sm.cand[slot];
+    const bool live = slot_live(sm, i);
+    const unsigned long long K = live ? sm.cand[i * RT + threadIdx.x] : 0ull;
     const float v = ckey_value(K);
-    if (bin0(v, m) != b) continue;
-    const double q = qmass(sm, v, m);
+    const bool in = live && bin0(v, m) == b;
+    const double q = in ? qmass(sm, v, m) : 0.0;
+    const bool kept = in && (uint32_t)(K >> 32) >= kt;
     ms += q;
-    ++c;
-    if ((uint32_t)(K >> 32) >= kt) {
-      km += q;
-      ++kc;
-      kmn = K < kmn ? K : kmn;
-    }
+    c += in ? 1 : 0;
+    km += kept ? q : 0.0;
+    kc += kept ? 1 : 0;
+    kmn = (kept && K < kmn) ? K : kmn;
   }
-  mass = block_sum_d(ms, sm);
-  cnt = block_sum_l(c, sm);
-  kept_mass = block_sum_d(km, sm);
-  kept_cnt = block_sum_l(kc, sm);
+  double v[4] = {ms, (double)c, km, (double)kc};  // counts are exact in a double
+  block_sum_multi<4>(v, sm);
+  mass = v[0];
+  cnt = (long long)v[1];
+  kept_mass = v[2];
+  kept_cnt = (long long)v[3];
   k_min = block_ext_u<false>(kmn, sm);
 }
 
@@ -943,23 +1078,19 @@ __device__ __noinline__ void gathered_bucket_stats(RSmem& sm, float m, int b, ui
 __device__ __noinline__ void window_stats(RSmem& sm, float m, int lo, int hi, double (&wm)[3],
                                           long long (&wc)[3]) {
   constexpr int PER = CAP / RT;
-  const int base = (int)threadIdx.x * PER;
-  const int wcnt = sm.wcount[base / WCAP];
   double ms[3] = {0.0, 0.0, 0.0};
   long long c[3] = {0, 0, 0};
+#pragma unroll 4
   for (int i = 0; i < PER; ++i) {
-    const int slot = base + i;
-    if ((slot % WCAP) >= wcnt) continue;
-    const float v = ckey_value(sm.cand[slot]);
-    const int b = bin0(v, m);
-    if (b < lo || b > hi) continue;
-    const double q = qmass(sm, v, m);
+    const bool live = slot_live(sm, i);
+    const float v = ckey_value(live ? sm.cand[i * RT + threadIdx.x] : 0ull);
+    const int w = live ? bin0(v, m) - lo : -1;
+    const double q = (w >= 0 && w <= hi - lo) ? qmass(sm, v, m) : 0.0;
 #pragma unroll
-    for (int w = 0; w < 3; ++w)
-      if (b - lo == w) {
-        ms[w] += q;
-        ++c[w];
-      }
+    for (int u = 0; u < 3; ++u) {
+      ms[u] += w == u ? q : 0.0;
+      c[u] += w == u ? 1 : 0;
+    }
   }
   double v[6] = {ms[0], ms[1], ms[2], (double)c[0], (double)c[1], (double)c[2]};
   block_sum_multi<6>(v, sm);
@@ -976,6 +1107,63 @@ __device__ int prev_nonempty(RSmem& sm, int b) {
   for (int i = threadIdx.x; i < b; i += RT)
     if (sm.cnt[i] > 0) mine = i;
   return (int)block_ext_u<true>((unsigned long long)(mine + 1), sm) - 1;
+}
+
+// The estimated top-p crossing bucket from the counts alone (every element
+// weighted by its bucket's mid-point mass; the far-tail bucket by 0): the first
+// non-empty bucket whose inclusive estimated mass reaches p * Zhat. Returns it
+// with the exact count of the elements before it.
+__device__ __noinline__ void plan_top_p(RSmem& sm, float p, int& b_out, long long& cnt_before) {
+  constexpr int PER = NB / RT;
+  const int base = (int)threadIdx.x * PER;
+  const double wmid = sm.bd[3];
+  int c[PER];
+  double q[PER];
+  long long lc = 0;
+  double lm = 0.0;
+  int last_nz = -1;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int b = base + i;
+    c[i] = sm.cnt[b];
+    q[i] = b < NB - 1 ? (double)c[i] * tab_at(sm.tab, b) * wmid : 0.0;
+    lc += c[i];
+    lm += q[i];
+    if (c[i] > 0) last_nz = b;
+  }
+  long long tc;
+  double tm;
+  long long pc;
+  double pm;
+  block_exscan2(lc, lm, pc, pm, tc, tm, sm);
+  const double target = (double)p * tm;
+  int mine = NB;
+  long long mine_before = 0;
+  {
+    long long cc = pc;
+    double ms = pm;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const long long before = cc;
+      cc += c[i];
+      ms += q[i];
+      if (mine == NB && c[i] > 0 && ms >= target) {
+        mine = base + i;
+        mine_before = before;
+      }
+    }
+  }
+  int b = block_min_i(mine, sm);
+  if (b >= NB) {  // rounding kept every estimate below the target: the last non-empty bucket
+    b = (int)block_ext_u<true>((unsigned long long)(unsigned)(last_nz + 1), sm) - 1;
+    if (threadIdx.x == 0) sm.bl[0] = tc - sm.cnt[b];
+  } else if (mine == b) {
+    sm.bl[0] = mine_before;
+  }
+  __syncthreads();
+  b_out = b;
+  cnt_before = sm.bl[0];
+  __syncthreads();
 }
 
 // Resolve a row with one count pass and one exact pass. Returns false when the
@@ -1012,13 +1200,13 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
     pick_bucket(sm, kCount, (long long)k, 0.0, 0, 0.0, bk, ce, me);
     const long long incl = ce + sm.cnt[bk];
     __syncthreads();
-    if (incl > CAP / 2) return false;  // keep the per-warp slices far from full
+    if (incl > SCAP) return false;  // keep the per-warp slices far from full
     pl.g_lo = 0;
     pl.g_hi = bk;
     pass2<VEC>(sm, x, V, m, false, pl, P);
     if (P.overflow) return false;
     const int n = compact_gathered(sm, m, 0, bk);
-    sort_and_scan(sm, 0, n, m);
+    sort_and_scan(sm, n, m);
     const int jk = min(k, n) - 1;
     Cut ck{sm.cand[jk], (long long)jk + 1, sm.cq[jk]};
     best = ck;
@@ -1044,20 +1232,14 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
   int lo = 0, hi = -1, bm = -1, bprev = -1;
   long long gathered = 0;
   if (p_on) {
-    for (int i = threadIdx.x; i < NB; i += RT)
-      sm.mass[i] = i < NB - 1 ? (double)sm.cnt[i] * sm.tab[i] * sm.bd[3] : 0.0;
-    __syncthreads();
-    double zl = 0.0;
-    for (int i = threadIdx.x; i < NB; i += RT) zl += sm.mass[i];
-    const double zhat = block_sum_d(zl, sm);
     int bh;
-    long long ce;
-    double me;
-    pick_bucket(sm, kMassGE, 0, (double)p * zhat, 0, 0.0, bh, ce, me);
+    long long cb;
+    plan_top_p(sm, p, bh, cb);
     lo = bh > 0 ? bh - 1 : 0;
     hi = bh < NB - 1 ? bh + 1 : NB - 1;
-    gathered += count_range(sm, lo, hi + 1);
-    before_win = count_range(sm, 0, lo);
+    const long long c_lo = lo < bh ? sm.cnt[lo] : 0, c_hi = hi > bh ? sm.cnt[hi] : 0;
+    gathered += c_lo + sm.cnt[bh] + c_hi;
+    before_win = cb - c_lo;
     pl.g_lo = lo;
     pl.g_hi = hi;
     pl.w_lo = lo;
@@ -1067,13 +1249,13 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
     bprev = prev_nonempty(sm, bm);
     before_mu = count_range(sm, 0, bm);
     const int a0 = bprev >= 0 ? bprev : bm;
-    gathered += count_range(sm, a0, bm + 1);
+    gathered += sm.cnt[bm] + (a0 < bm ? sm.cnt[a0] : 0);  // buckets between are empty
     pl.g2_lo = a0;
     pl.g2_hi = bm;
     pl.b_mu = bm;
   }
   __syncthreads();
-  if (gathered > CAP / 2) return false;  // keep the per-warp slices far from full
+  if (gathered > SCAP) return false;  // keep the per-warp slices far from full
   pass2<VEC>(sm, x, V, m, p_on, pl, P);
   if (P.overflow) return false;
 
@@ -1111,7 +1293,7 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
     }
     if (c < 0) return false;  // the crossing lies outside the window
     const int n = compact_gathered(sm, m, c, c);
-    sort_and_scan(sm, 0, n, m);
+    sort_and_scan(sm, n, m);
     const int jp = first_mass_hit(sm, 0, n, before, 0.0, kMassGE, target);
     const Cut cp{sm.cand[jp], cbefore + jp + 1, before + sm.cq[jp]};
     if (have)
@@ -1128,13 +1310,42 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   RSmem& sm = *reinterpret_cast<RSmem*>(smem_raw);
   const int V = a.V;
-  for (int i = threadIdx.x; i < NB; i += RT) sm.tab[i] = exp(-(double)i * (1.0 / 128.0));
+  init_exp_tab(sm.tab, threadIdx.x, RT);
   if (threadIdx.x == 0) sm.bd[3] = exp(-1.0 / 256.0);  // mid-bucket weight factor
   __syncthreads();
 
+  // A row's metadata and the first two of its partial maxima per thread are
+  // loaded one row ahead, so their latency overlaps the previous row's work.
+  struct Ahead {
+    float part0, part1, p, mu;
+    int flags, k;
+  };
+  auto load_ahead = [&](int row, Ahead& h) {
+    h.part0 = h.part1 = -INFINITY;
+    h.flags = 0;
+    h.k = 0;
+    h.p = 1.0f;
+    h.mu = 0.0f;
+    if (row >= a.rows) return;
+    if (a.max_part) {
+      const float* mp = a.max_part + (size_t)row * (size_t)a.n_parts;
+      const int i0 = threadIdx.x, i1 = threadIdx.x + RT;
+      if (i0 < a.n_parts) h.part0 = mp[i0];
+      if (i1 < a.n_parts) h.part1 = mp[i1];
+    }
+    if (a.row_flags) h.flags = a.row_flags[row];
+    h.k = a.top_k[row];
+    h.p = a.top_p[row];
+    h.mu = a.min_p[row];
+  };
+  Ahead ahead;
+  load_ahead(blockIdx.x, ahead);
+
   for (int r = blockIdx.x; r < a.rows; r += gridDim.x) {
+    const Ahead cur = ahead;
+    load_ahead(r + gridDim.x, ahead);
     const float* __restrict__ x = a.S + (size_t)r * (size_t)a.ld;
-    const bool invalid = a.row_flags && (a.row_flags[r] & STS_ROW_INVALID);
+    const bool invalid = (cur.flags & STS_ROW_INVALID) != 0;
     if (invalid) {
       if (threadIdx.x == 0) {
         const float nan = __int_as_float(0x7fc00000);
@@ -1157,16 +1368,17 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
     float lm = -INFINITY;
     if (a.max_part) {
       const float* mp = a.max_part + (size_t)r * (size_t)a.n_parts;
-      for (int i = threadIdx.x; i < a.n_parts; i += RT) lm = fmaxf(lm, mp[i]);
+      lm = fmaxf(cur.part0, cur.part1);
+      for (int i = threadIdx.x + 2 * RT; i < a.n_parts; i += RT) lm = fmaxf(lm, mp[i]);
     } else {
       lm = row_max_pass<VEC>(x, V);
     }
     const float m = block_max_f(lm, sm);
     const double md = (double)m;
 
-    const int k = a.top_k[r];
-    const float p = a.top_p[r];
-    const float mu = a.min_p[r];
+    const int k = cur.k;
+    const float p = cur.p;
+    const float mu = cur.mu;
     const bool k_on = k >= 1 && k < V;
     const bool p_on = p < 1.0f;
     const bool mu_on = mu > 0.0f;
@@ -1259,8 +1471,8 @@ __global__ void validate_kernel(const int64_t* target, const float* temperature,
 // Evaluates the resolver's mass function exp(s - m) and the library exp on
 // the same inputs (test hook for the table-driven exponential).
 __global__ void mass_probe_kernel(const float* s, float m, double* mine, double* lib, int64_t n) {
-  __shared__ double tab[NB];
-  for (int i = threadIdx.x; i < NB; i += blockDim.x) tab[i] = exp(-(double)i * (1.0 / 128.0));
+  __shared__ ExpTab tab;
+  init_exp_tab(tab, threadIdx.x, blockDim.x);
   __syncthreads();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -1280,6 +1492,10 @@ void launch_validate(const int64_t* target, const float* temperature, const floa
   validate_kernel<<<blocks, threads, 0, stream>>>(target, temperature, top_p, min_p, T, V, flags,
                                                   hdr, check_target ? 1 : 0);
 }
+
+static_assert(sizeof(RSmem) <= 227 * 1024, "the resolver CTA fits one SM's shared memory");
+static_assert(NB == SCAP, "bucket masses and the candidates' scan share storage");
+static_assert(SCAP <= CAP && SCAP == 8 * RT, "a sorted run fits the candidate buffer");
 
 size_t resolve_smem_bytes() { return sizeof(RSmem); }
 
