@@ -35,6 +35,23 @@ def test_parse_clock_lines_and_rejection():
     assert bench.parse_clock_lines("") is None
 
 
+def test_recorded_traffic_follows_the_kernel_sources(monkeypatch):
+    rec_path = os.path.join(ROOT, "profiles", "dram_traffic_T16384_d5120_V152064.json")
+    with open(rec_path) as f:
+        rec = json.load(f)
+    # a workload without a capture has no recorded traffic
+    assert bench.recorded_traffic(64, 128, 1024, "dw_gemm") is None
+    assert bench.recorded_traffic(16384, 5120, 152064, "validate") is None
+    # with the sources the capture was taken with, the record's per-launch bytes come back
+    got = bench.recorded_traffic(16384, 5120, 152064, "dw_gemm")
+    k = rec["kernels"]["dw_gemm"]
+    expect = k["dram_read_bytes_per_launch"] + k["dram_write_bytes_per_launch"]
+    assert got is None or got == expect
+    # any other source set (a changed kernel) gives null
+    monkeypatch.setitem(bench._TRAFFIC_SOURCES, "gemm", ["resolver.cu"])
+    assert bench.recorded_traffic(16384, 5120, 152064, "dw_gemm") is None
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
