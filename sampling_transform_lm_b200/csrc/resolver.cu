@@ -55,6 +55,7 @@
 // degree-6 Taylor polynomial, whose truncation error (< 4e-19) is below half
 // an ulp. Elements in the clamped far-tail bucket use the library exp.
 #include <cfloat>
+#include <type_traits>
 #include <cmath>
 
 #include "sts_device.cuh"
@@ -129,11 +130,14 @@ __device__ __forceinline__ int ckey_id(unsigned long long K) {
   return (int)(0xFFFFFFFFu - (uint32_t)(K & 0xFFFFFFFFull));
 }
 
+// Level-0 bucket of s: floor((m - s) * 128) clamped to [0, NB - 1]. The floor
+// takes no conversion instruction: adding 2^23 rounding toward -inf leaves
+// floor(f) in the low mantissa bits (f < 2^23, one unit per ulp).
 __device__ __forceinline__ int bin0(float s, float m) {
-  const float f = fminf((m - s) * BIN_SCALE, (float)(NB - 1));
-  const int b = (int)f;
-  return b < 0 ? 0 : b;
+  const float f = fminf(fmaxf((m - s) * BIN_SCALE, 0.0f), (float)(NB - 1));
+  return __float_as_int(__fadd_rd(f, 8388608.0f)) - 0x4B000000;
 }
+
 
 // exp(x) for the far tail (x < -32), kept out of line so the loops that
 // stream a row do not carry its registers.
@@ -143,7 +147,7 @@ __device__ __noinline__ double far_mass(double x) { return exp(x); }
 __device__ __forceinline__ double qmass_b(const ExpTab& tab, float s, double md, int b) {
   const double x = (double)s - md;
   if (b >= NB - 1) return far_mass(x);
-  const double r = x + (double)b * (1.0 / 128.0);
+  const double r = fma((double)b, 1.0 / 128.0, x);
   double p = 1.0 / 720.0;
   p = fma(p, r, 1.0 / 120.0);
   p = fma(p, r, 1.0 / 24.0);
@@ -170,6 +174,28 @@ __device__ __forceinline__ float4 ld_stream4(const float4* p) {
   return v;
 }
 
+// L2 eviction policies for the two passes over a row: the count pass marks
+// the row's lines evict-last so the exact pass that follows finds them in L2
+// (148 rows in flight are about 90 MB), and the exact pass reads them
+// evict-first, which hands the space back.
+__device__ __forceinline__ unsigned long long l2_policy_keep() {
+  unsigned long long p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ unsigned long long l2_policy_drop() {
+  unsigned long long p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ float4 ld_stream4(const float4* p, unsigned long long policy) {
+  float4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p), "l"(policy));
+  return v;
+}
+
 __device__ __forceinline__ float ld_stream(const float* p) {
   float v;
   asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
@@ -178,17 +204,18 @@ __device__ __forceinline__ float ld_stream(const float* p) {
 
 // Apply f(value, index) to every element of the row. VEC: the row start is
 // 16-byte aligned, so UNROLL float4 loads per thread are kept in flight.
-template <bool VEC, typename F>
+template <bool VEC, bool KEEP = false, typename F>
 __device__ __forceinline__ void for_each(const float* __restrict__ x, int V, F&& f) {
   if (VEC) {
     const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
     const int V4 = V >> 2;
+    const unsigned long long keep = KEEP ? l2_policy_keep() : 0ull;
     for (int base = 0; base < V4; base += RT * UNROLL) {
       float4 v[UNROLL];
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
         const int i = base + u * RT + (int)threadIdx.x;
-        if (i < V4) v[u] = ld_stream4(x4 + i);
+        if (i < V4) v[u] = KEEP ? ld_stream4(x4 + i, keep) : ld_stream4(x4 + i);
       }
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
@@ -828,7 +855,7 @@ template <bool VEC>
 __device__ __noinline__ void count_hist(RSmem& sm, const float* __restrict__ x, int V, float m) {
   for (int i = threadIdx.x; i < NB; i += RT) sm.cnt[i] = 0;
   __syncthreads();
-  for_each<VEC>(x, V, [&](float s, int) { atomicAdd(&sm.cnt[bin0(s, m)], 1); });
+  for_each<VEC, true>(x, V, [&](float s, int) { atomicAdd(&sm.cnt[bin0(s, m)], 1); });
   __syncthreads();
 }
 
@@ -886,8 +913,6 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
   constexpr int E = 8;
   const double md = (double)m;
   const bool need_last = pl.need_last != 0;
-  // bucket ranges as (start, span) for one unsigned compare each; an empty
-  // range starts past the last bucket
   const int g_lo = pl.g_lo, g_hi = pl.g_hi, g2_lo = pl.g2_lo, g2_hi = pl.g2_hi;
   const int w_lo = pl.w_lo, b_mu = pl.b_mu;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -898,14 +923,18 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
   unsigned long long kl = ~0ull;
 
   // Element e < 4 of a batch is token a0 + e (valid when e < na), element
-  // e >= 4 is token b0 + e - 4 (valid when e - 4 < nb). The body has no
-  // per-element branches: masses are computed for all E elements and
-  // selected, the far tail (bucket NB - 1) takes one warp vote per batch, and
-  // each gather store is predicated on its ballot rather than branched over.
+  // e >= 4 is token b0 + e - 4 (valid when e - 4 < nb); `full` (a type)
+  // states at compile time that all are valid, which holds for every sweep
+  // but the last. The body has no per-element branches: masses are computed
+  // for all E elements and selected, the far tail (bucket NB - 1) takes one
+  // warp vote per batch, the gather votes run only when some lane of the warp
+  // has an element to gather, and each gather store is predicated on its
+  // ballot rather than branched over.
   const bool need_mass = NEED_Z || b_mu >= 0;
-  auto batch = [&](const float (&sv)[E], int a0, int na, int b0, int nb) {
+  const bool need_mu = b_mu >= 0;
+  auto batch = [&](auto full, const float (&sv)[E], int a0, int na, int b0, int nb) {
     auto idx = [&](int e) { return e < 4 ? a0 + e : b0 + (e - 4); };
-    auto ok = [&](int e) { return e < 4 ? e < na : e - 4 < nb; };
+    auto ok = [&](int e) { return decltype(full)::value || (e < 4 ? e < na : e - 4 < nb); };
     int bb[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) bb[e] = bin0(sv[e], m);
@@ -932,14 +961,16 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
           if (bb[e] >= NB - 1) qq[e] = far_mass((double)sv[e] - md);
       }
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const double q = ok(e) ? qq[e] : 0.0;
-        if (NEED_Z) {
-          z[e & 1] += q;
-          ap[e & 1] += bb[e] < w_lo ? q : 0.0;
+      for (int e = 0; e < E; ++e) qq[e] = ok(e) ? qq[e] : 0.0;
+      if (NEED_Z)
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          z[e & 1] += qq[e];
+          ap[e & 1] += bb[e] < w_lo ? qq[e] : 0.0;
         }
-        amu[e & 1] += bb[e] < b_mu ? q : 0.0;
-      }
+      if (need_mu)
+#pragma unroll
+        for (int e = 0; e < E; ++e) amu[e & 1] += bb[e] < b_mu ? qq[e] : 0.0;
     }
     if (need_last) {
 #pragma unroll
@@ -948,14 +979,22 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
         kl = K < kl ? K : kl;
       }
     }
+    unsigned gm = 0;  // this thread's elements in a gathered range, one bit each
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const int b = bb[e];
       const bool g = ok(e) && ((b >= g_lo && b <= g_hi) || (b >= g2_lo && b <= g2_hi));
-      const unsigned mk = __ballot_sync(0xffffffffu, g);
-      const int slot = wfill + __popc(mk & lt);
-      if (g && slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
-      wfill += __popc(mk);
+      gm |= g ? 1u << e : 0u;
+    }
+    if (__any_sync(0xffffffffu, gm != 0u)) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const bool g = (gm >> e) & 1u;
+        const unsigned mk = __ballot_sync(0xffffffffu, g);
+        const int slot = wfill + __popc(mk & lt);
+        if (g && slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
+        wfill += __popc(mk);
+      }
     }
   };
 
@@ -967,20 +1006,27 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
     // pairs two of those float4s.
     const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
     const int V4 = V >> 2;
-    for (int base = 0; base < V4; base += RT * 4) {
+    const unsigned long long drop = l2_policy_drop();
+    const int full_end = V4 - V4 % (RT * 4);  // sweeps where every thread's loads are in the row
+    for (int base = 0; base < full_end; base += RT * 4) {
       float4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + u * RT + tid;
-        v[u] = i < V4 ? ld_stream4(x4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      for (int u = 0; u < 4; ++u) v[u] = ld_stream4(x4 + base + u * RT + tid, drop);
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         const int ia = base + 2 * h * RT + tid, ib = ia + RT;
         const float4 a4 = h ? v[2] : v[0], b4 = h ? v[3] : v[1];
         const float sv[E] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
-        batch(sv, 4 * ia, ia < V4 ? 4 : 0, 4 * ib, ib < V4 ? 4 : 0);
+        batch(std::true_type{}, sv, 4 * ia, 4, 4 * ib, 4);
       }
+    }
+    for (int base = full_end; base < V4; base += RT * 2) {  // the last partial sweep
+      const int ia = base + tid, ib = ia + RT;
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 a4 = ia < V4 ? ld_stream4(x4 + ia, drop) : z4;
+      const float4 b4 = ib < V4 ? ld_stream4(x4 + ib, drop) : z4;
+      const float sv[E] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+      batch(std::false_type{}, sv, 4 * ia, ia < V4 ? 4 : 0, 4 * ib, ib < V4 ? 4 : 0);
     }
     tail0 = 4 * V4;
   }
@@ -989,7 +1035,7 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
     const bool in = i < V;
     const float t = in ? ld_stream(x + i) : 0.f;
     const float sv[E] = {t, t, t, t, t, t, t, t};
-    batch(sv, i, in ? 1 : 0, i, 0);
+    batch(std::false_type{}, sv, i, in ? 1 : 0, i, 0);
   }
   if (lane == 0) sm.wcount[warp] = wfill;
   double sums[3] = {z[0] + z[1], ap[0] + ap[1], amu[0] + amu[1]};
