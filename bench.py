@@ -337,6 +337,17 @@ def run_ours(args, rank, local_rank, world):
                 "traffic": recorded_traffic(T, d, V, dom), "launches": dom_n,
                 "ms_per_step": round(dom_ms / args.steps, 3)}
     per_kernel = {n: round(v[0] / args.steps, 3) for n, v in kern.items() if v[1]}
+    # the resolver against HBM whether or not it dominates: one read of the
+    # row chunks' fp32 logits per step is its algorithmic traffic
+    res_ms, res_n = kern.get("resolve", (0.0, 0))
+    roof_res = None
+    if res_n:
+        gbs = 4.0 * T * V * args.steps / (res_ms / 1e3) / 1e9
+        roof_res = {"kernel": "resolve", "bound": "hbm", "achieved": round(gbs, 1),
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                    "traffic": recorded_traffic(T, d, V, "resolve"), "launches": res_n,
+                    "ms_per_step": round(res_ms / args.steps, 3),
+                    "note": "issue-bound (float64-exact masses); see profiles/resolve_kernel_*.md"}
 
     # end to end through the public API: inputs from pinned host memory, the
     # step's logprobs read back every step (W stays resident: a model weight)
@@ -412,6 +423,7 @@ def run_ours(args, rank, local_rank, world):
                         "runs one GEMM pass and resolves on stored fp32 logits",
             },
             "roofline": roof,
+            "roofline_resolver": roof_res,
             "kernel_ms_per_step": per_kernel,
             "e2e": {"value": round(world * T / (e2e_ms / 1e3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
