@@ -408,7 +408,7 @@ def run_ours(args, rank, local_rank, world):
                     f" [reduced to T={T}, V={V} for a profiling capture]"
                     if (args.rows or args.vocab) else ""),
                 "T_per_gpu": T, "d": d, "V": V, "global_batch": world * T,
-                "vocab_chunk": wl.vocab_chunk or 16384,
+                "vocab_chunk": sts.sts_vocab_chunk(T, d, V, wl.vocab_chunk),
                 "parallelism": f"dp{world} (one batch per GPU, no collective on the data path)",
                 "l2": "inputs larger than L2 (W alone is %.2f GB)" % (V * d * 2 / 1e9),
             },

@@ -26,6 +26,7 @@ __all__ = [
     "load",
     "library_path",
     "sts_workspace_bytes",
+    "sts_vocab_chunk",
     "sts_forward",
     "sts_backward",
     "sts_sample",
@@ -61,6 +62,7 @@ KERNEL_KINDS = ("validate", "logits_gemm", "resolve", "dz_gemm", "dw_gemm", "dh_
 
 EXPORTED_SYMBOLS = (
     "sts_workspace_bytes",
+    "sts_vocab_chunk",
     "sts_forward",
     "sts_backward",
     "sts_sample",
@@ -120,6 +122,8 @@ def load():
     P, S, I64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64
     lib.sts_workspace_bytes.argtypes = [ctypes.POINTER(_Shape), ctypes.c_int]
     lib.sts_workspace_bytes.restype = S
+    lib.sts_vocab_chunk.argtypes = [ctypes.POINTER(_Shape)]
+    lib.sts_vocab_chunk.restype = ctypes.c_int64
     lib.sts_forward.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows), P,
                                 ctypes.POINTER(_Saved), P, S, P]
     lib.sts_forward.restype = ctypes.c_int
@@ -215,6 +219,16 @@ def sts_workspace_bytes(T, d, V, pass_, vocab_chunk=0, row_chunk=0) -> int:
     n = load().sts_workspace_bytes(ctypes.byref(sh), int(pass_))
     if n == 0:
         raise StsError(STS_ERR_SHAPE, "sts_workspace_bytes")
+    return int(n)
+
+
+def sts_vocab_chunk(T, d, V, vocab_chunk=0) -> int:
+    """The backward's vocabulary chunk for this shape (the automatic choice
+    when ``vocab_chunk`` is 0)."""
+    sh = _shape(T, d, V, vocab_chunk, 0)
+    n = load().sts_vocab_chunk(ctypes.byref(sh))
+    if n < 0:
+        raise StsError(STS_ERR_SHAPE, "sts_vocab_chunk")
     return int(n)
 
 
