@@ -377,47 +377,45 @@ __device__ T block_exscan(T v, T* warp_tot, T& total) {
   return before_warp + x - v;
 }
 
-// Exclusive scans of a count and a mass over threads in thread order, in one
+// Exclusive scans of three doubles over threads in thread order, in one
 // exchange.
-__device__ void block_exscan2(long long a, double b, long long& pa, double& pb, long long& ta,
-                              double& tb, RSmem& sm) {
+__device__ void block_exscan_d3(const double (&v)[3], double (&pre)[3], double (&tot)[3], RSmem& sm) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  long long xa = a;
-  double xb = b;
+  double x[3] = {v[0], v[1], v[2]};
   for (int o = 1; o < 32; o <<= 1) {
-    const long long ya = __shfl_up_sync(0xffffffffu, xa, o);
-    const double yb = __shfl_up_sync(0xffffffffu, xb, o);
-    if (l >= o) {
-      xa += ya;
-      xb += yb;
-    }
+    double y[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) y[k] = __shfl_up_sync(0xffffffffu, x[k], o);
+    if (l >= o)
+#pragma unroll
+      for (int k = 0; k < 3; ++k) x[k] += y[k];
   }
-  if (l == 31) {
-    sm.red_l[w] = xa;
-    sm.red_d[w] = xb;
-  }
+  if (l == 31)
+#pragma unroll
+    for (int k = 0; k < 3; ++k) sm.red_m[w * 8 + k] = x[k];
   __syncthreads();
   if (w == 0) {
-    long long s = l < NWARP ? sm.red_l[l] : 0;
-    double d = l < NWARP ? sm.red_d[l] : 0.0;
+    double t[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) t[k] = l < NWARP ? sm.red_m[l * 8 + k] : 0.0;
     for (int o = 1; o < 32; o <<= 1) {
-      const long long ys = __shfl_up_sync(0xffffffffu, s, o);
-      const double yd = __shfl_up_sync(0xffffffffu, d, o);
-      if (l >= o) {
-        s += ys;
-        d += yd;
-      }
+      double y[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) y[k] = __shfl_up_sync(0xffffffffu, t[k], o);
+      if (l >= o)
+#pragma unroll
+        for (int k = 0; k < 3; ++k) t[k] += y[k];
     }
-    if (l < NWARP) {
-      sm.red_l[l] = s;  // inclusive warp prefixes
-      sm.red_d[l] = d;
-    }
+    if (l < NWARP)
+#pragma unroll
+      for (int k = 0; k < 3; ++k) sm.red_m[l * 8 + k] = t[k];  // inclusive warp prefixes
   }
   __syncthreads();
-  pa = (w > 0 ? sm.red_l[w - 1] : 0) + xa - a;
-  pb = (w > 0 ? sm.red_d[w - 1] : 0.0) + xb - b;
-  ta = sm.red_l[NWARP - 1];
-  tb = sm.red_d[NWARP - 1];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    pre[k] = (w > 0 ? sm.red_m[(w - 1) * 8 + k] : 0.0) + x[k] - v[k];
+    tot[k] = sm.red_m[(NWARP - 1) * 8 + k];
+  }
   __syncthreads();
 }
 
@@ -1158,58 +1156,74 @@ __device__ int prev_nonempty(RSmem& sm, int b) {
 // The estimated top-p crossing bucket from the counts alone (every element
 // weighted by its bucket's mid-point mass; the far-tail bucket by 0): the first
 // non-empty bucket whose inclusive estimated mass reaches p * Zhat. Returns it
-// with the exact count of the elements before it.
-__device__ __noinline__ void plan_top_p(RSmem& sm, float p, int& b_out, long long& cnt_before) {
+// with the exact count of the elements before it, the estimated masses before
+// it (e0) and of it (eb), Zhat, and sigma, the standard deviation of the
+// estimate's error were the elements spread uniformly within their buckets
+// (per element sd(exp(r)) = 0.00226 exp(-b / 128) for r uniform on a bucket).
+struct TopPPlan {
+  int b;
+  long long cnt_before;
+  double e0, eb, zhat, sigma;
+};
+
+__device__ __noinline__ TopPPlan plan_top_p(RSmem& sm, float p) {
   constexpr int PER = NB / RT;
+  constexpr double kSdPerElement = 0.0022552;  // sd of exp(r), r ~ U(-1/128, 0]
   const int base = (int)threadIdx.x * PER;
   const double wmid = sm.bd[3];
   int c[PER];
   double q[PER];
-  long long lc = 0;
-  double lm = 0.0;
+  double loc[3] = {0.0, 0.0, 0.0};  // count, estimated mass, error variance
   int last_nz = -1;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int b = base + i;
     c[i] = sm.cnt[b];
-    q[i] = b < NB - 1 ? (double)c[i] * tab_at(sm.tab, b) * wmid : 0.0;
-    lc += c[i];
-    lm += q[i];
+    const double t = b < NB - 1 ? tab_at(sm.tab, b) : 0.0;
+    q[i] = (double)c[i] * t * wmid;
+    loc[0] += c[i];
+    loc[1] += q[i];
+    loc[2] += (double)c[i] * (t * kSdPerElement) * (t * kSdPerElement);
     if (c[i] > 0) last_nz = b;
   }
-  long long tc;
-  double tm;
-  long long pc;
-  double pm;
-  block_exscan2(lc, lm, pc, pm, tc, tm, sm);
-  const double target = (double)p * tm;
+  double pre[3], tot[3];
+  block_exscan_d3(loc, pre, tot, sm);
+  const double target = (double)p * tot[1];
   int mine = NB;
-  long long mine_before = 0;
+  double mine_before = 0.0, mine_e0 = 0.0, mine_eb = 0.0;
   {
-    long long cc = pc;
-    double ms = pm;
+    double cc = pre[0], ms = pre[1];
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-      const long long before = cc;
+      const double before = cc, e0 = ms;
       cc += c[i];
       ms += q[i];
       if (mine == NB && c[i] > 0 && ms >= target) {
         mine = base + i;
         mine_before = before;
+        mine_e0 = e0;
+        mine_eb = q[i];
       }
     }
   }
   int b = block_min_i(mine, sm);
   if (b >= NB) {  // rounding kept every estimate below the target: the last non-empty bucket
     b = (int)block_ext_u<true>((unsigned long long)(unsigned)(last_nz + 1), sm) - 1;
-    if (threadIdx.x == 0) sm.bl[0] = tc - sm.cnt[b];
+    if (threadIdx.x == 0) {
+      const double eb = (double)sm.cnt[b] * (b < NB - 1 ? tab_at(sm.tab, b) : 0.0) * wmid;
+      sm.bd[0] = tot[0] - sm.cnt[b];
+      sm.bd[1] = tot[1] - eb;
+      sm.bd[2] = eb;
+    }
   } else if (mine == b) {
-    sm.bl[0] = mine_before;
+    sm.bd[0] = mine_before;
+    sm.bd[1] = mine_e0;
+    sm.bd[2] = mine_eb;
   }
   __syncthreads();
-  b_out = b;
-  cnt_before = sm.bl[0];
+  TopPPlan pl{b, (long long)sm.bd[0], sm.bd[1], sm.bd[2], tot[1], sqrt(tot[2])};
   __syncthreads();
+  return pl;
 }
 
 // Resolve a row with one count pass and one exact pass. Returns false when the
@@ -1272,83 +1286,96 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
   }
 
   // top-k off: estimate the top-p crossing bucket from counts x mid-bucket
-  // weights and gather a 3-bucket window around it; for min-p gather the
-  // threshold's bucket and the non-empty bucket before it
-  long long before_win = 0, before_mu = 0;
-  int lo = 0, hi = -1, bm = -1, bprev = -1;
-  long long gathered = 0;
-  if (p_on) {
-    int bh;
-    long long cb;
-    plan_top_p(sm, p, bh, cb);
-    lo = bh > 0 ? bh - 1 : 0;
-    hi = bh < NB - 1 ? bh + 1 : NB - 1;
-    const long long c_lo = lo < bh ? sm.cnt[lo] : 0, c_hi = hi > bh ? sm.cnt[hi] : 0;
-    gathered += c_lo + sm.cnt[bh] + c_hi;
-    before_win = cb - c_lo;
-    pl.g_lo = lo;
-    pl.g_hi = hi;
-    pl.w_lo = lo;
-  }
-  if (mu_on) {
-    bm = bin0(key32_value(kt), m);
-    bprev = prev_nonempty(sm, bm);
-    before_mu = count_range(sm, 0, bm);
-    const int a0 = bprev >= 0 ? bprev : bm;
-    gathered += sm.cnt[bm] + (a0 < bm ? sm.cnt[a0] : 0);  // buckets between are empty
-    pl.g2_lo = a0;
-    pl.g2_hi = bm;
-    pl.b_mu = bm;
-  }
-  __syncthreads();
-  if (gathered > SCAP) return false;  // keep the per-warp slices far from full
-  pass2<VEC>(sm, x, V, m, p_on, pl, P);
-  if (P.overflow) return false;
+  // weights and gather it, with a neighbour bucket on each side where the
+  // estimate comes within six sigma (plus 1e-5 Zhat for bias) of the target;
+  // if the exact masses then put the crossing outside, retry once with the
+  // full 3-bucket window. For min-p gather the threshold's bucket and the
+  // non-empty bucket before it.
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    long long before_win = 0, before_mu = 0;
+    int lo = 0, hi = -1, bm = -1, bprev = -1;
+    bool narrowed = false;
+    long long gathered = 0;
+    if (p_on) {
+      const TopPPlan tp = plan_top_p(sm, p);
+      const int bh = tp.b;
+      const double t = (double)p * tp.zhat, margin = 6.0 * tp.sigma + 1e-5 * tp.zhat;
+      const bool near_lo = attempt > 0 || t - tp.e0 < margin;
+      const bool near_hi = attempt > 0 || tp.e0 + tp.eb - t < margin;
+      lo = (near_lo && bh > 0) ? bh - 1 : bh;
+      hi = (near_hi && bh < NB - 1) ? bh + 1 : bh;
+      narrowed = (bh > 0 && lo == bh) || (bh < NB - 1 && hi == bh);
+      const long long c_lo = lo < bh ? sm.cnt[lo] : 0, c_hi = hi > bh ? sm.cnt[hi] : 0;
+      gathered += c_lo + sm.cnt[bh] + c_hi;
+      before_win = tp.cnt_before - c_lo;
+      pl.g_lo = lo;
+      pl.g_hi = hi;
+      pl.w_lo = lo;
+    }
+    if (mu_on) {
+      bm = bin0(key32_value(kt), m);
+      bprev = prev_nonempty(sm, bm);
+      before_mu = count_range(sm, 0, bm);
+      const int a0 = bprev >= 0 ? bprev : bm;
+      gathered += sm.cnt[bm] + (a0 < bm ? sm.cnt[a0] : 0);  // buckets between are empty
+      pl.g2_lo = a0;
+      pl.g2_hi = bm;
+      pl.b_mu = bm;
+    }
+    __syncthreads();
+    if (gathered > SCAP) return false;  // keep the per-warp slices far from full
+    pass2<VEC>(sm, x, V, m, p_on, pl, P);
+    if (P.overflow) return false;
 
-  bool have = false;
-  if (mu_on) {
-    double mass, kmass;
-    long long cnt, kcnt;
-    unsigned long long kmin;
-    gathered_bucket_stats(sm, m, bm, kt, mass, cnt, kmass, kcnt, kmin);
-    if (kcnt == 0 && bprev >= 0) {
-      // nothing of bucket bm is kept: the min-p prefix ends with bucket bprev
-      double m2, k2;
-      long long c2, kc2;
-      gathered_bucket_stats(sm, m, bprev, 0u, m2, c2, k2, kc2, kmin);
-    }
-    best = Cut{kmin, before_mu + kcnt, P.a_mu + kmass};
-    have = true;
-  }
-  if (p_on) {
-    const double target = (double)p * P.z;
-    // the crossing bucket, from the exact masses of the gathered window
-    double wm[3];
-    long long wc[3];
-    window_stats(sm, m, lo, hi, wm, wc);
-    double before = P.a_p;
-    long long cbefore = before_win;
-    int c = -1;
-    for (int w = lo; w <= hi; ++w) {
-      if (before < target && target <= before + wm[w - lo]) {
-        c = w;
-        break;
+    bool have = false;
+    if (mu_on) {
+      double mass, kmass;
+      long long cnt, kcnt;
+      unsigned long long kmin;
+      gathered_bucket_stats(sm, m, bm, kt, mass, cnt, kmass, kcnt, kmin);
+      if (kcnt == 0 && bprev >= 0) {
+        // nothing of bucket bm is kept: the min-p prefix ends with bucket bprev
+        double m2, k2;
+        long long c2, kc2;
+        gathered_bucket_stats(sm, m, bprev, 0u, m2, c2, k2, kc2, kmin);
       }
-      before += wm[w - lo];
-      cbefore += wc[w - lo];
+      best = Cut{kmin, before_mu + kcnt, P.a_mu + kmass};
+      have = true;
     }
-    if (c < 0) return false;  // the crossing lies outside the window
-    const int n = compact_gathered(sm, m, c, c);
-    sort_and_scan(sm, n, m);
-    const int jp = first_mass_hit(sm, 0, n, before, 0.0, kMassGE, target);
-    const Cut cp{sm.cand[jp], cbefore + jp + 1, before + sm.cq[jp]};
-    if (have)
-      take_earlier(best, cp);
-    else
-      best = cp;
+    if (p_on) {
+      const double target = (double)p * P.z;
+      // the crossing bucket, from the exact masses of the gathered window
+      double wm[3];
+      long long wc[3];
+      window_stats(sm, m, lo, hi, wm, wc);
+      double before = P.a_p;
+      long long cbefore = before_win;
+      int c = -1;
+      for (int w = lo; w <= hi; ++w) {
+        if (before < target && target <= before + wm[w - lo]) {
+          c = w;
+          break;
+        }
+        before += wm[w - lo];
+        cbefore += wc[w - lo];
+      }
+      if (c < 0) {  // the crossing lies outside the window
+        if (narrowed) continue;
+        return false;
+      }
+      const int n = compact_gathered(sm, m, c, c);
+      sort_and_scan(sm, n, m);
+      const int jp = first_mass_hit(sm, 0, n, before, 0.0, kMassGE, target);
+      const Cut cp{sm.cand[jp], cbefore + jp + 1, before + sm.cq[jp]};
+      if (have)
+        take_earlier(best, cp);
+      else
+        best = cp;
+    }
+    __syncthreads();
+    return true;
   }
-  __syncthreads();
-  return true;
+  return false;
 }
 
 template <bool VEC>
