@@ -889,14 +889,6 @@ struct Plan2 {
 };
 
 constexpr int WCAP = CAP / NWARP;  // private gather slots per warp
-// Readers of the slices take slot i * RT + tid (i < CAP / RT), which is
-// position (i % SLR) * RT + tid of slice i / SLR: a warp reads 32 consecutive
-// keys (no bank conflicts).
-constexpr int SLR = WCAP / RT;  // reader steps per slice
-static_assert(WCAP % RT == 0, "a slice is a whole number of reader steps");
-__device__ __forceinline__ bool slot_live(const RSmem& sm, int i) {
-  return (i % SLR) * RT + (int)threadIdx.x < sm.wcount[i / SLR];
-}
 
 // One pass over the row: exact float64 masses accumulated in registers, and
 // the elements of up to two bucket ranges gathered into per-warp slices of
@@ -1057,56 +1049,73 @@ __device__ void pass2(RSmem& sm, const float* __restrict__ x, int V, float m, bo
     pass2_impl<VEC, false>(sm, x, V, m, pl, P);
 }
 
-// Move the gathered candidates whose bucket lies in [lo, hi] from the per-warp
-// slices to sm.cand[0, n) (block scan, order irrelevant: they are sorted
-// next). At most SCAP are kept. Returns n.
-__device__ __noinline__ int compact_gathered(RSmem& sm, float m, int lo, int hi) {
-  constexpr int PER = CAP / RT;
+// Packs the live keys of the per-warp slices densely, in slice order, into the
+// storage of sm.cq (free until the sort writes its scan), so the readers below
+// spread them over every thread. Returns their number (the plan bounds it by
+// SCAP).
+__device__ __forceinline__ unsigned long long* packed(RSmem& sm) {
+  return reinterpret_cast<unsigned long long*>(sm.cq);
+}
+
+__device__ __noinline__ int pack_gathered(RSmem& sm) {
+  unsigned long long* g = packed(sm);
+  int off = 0;
+  for (int w = 0; w < NWARP; ++w) {
+    const int cnt = min(sm.wcount[w], WCAP);
+    for (int j = threadIdx.x; j < cnt; j += RT)
+      if (off + j < SCAP) g[off + j] = sm.cand[w * WCAP + j];
+    off += cnt;
+  }
+  __syncthreads();
+  return min(off, SCAP);
+}
+
+// Move the n packed candidates whose bucket lies in [lo, hi] to
+// sm.cand[0, n') (block scan, order irrelevant: they are sorted next).
+// Returns n'.
+__device__ __noinline__ int compact_gathered(RSmem& sm, int n, float m, int lo, int hi) {
+  constexpr int PER = SCAP / RT;
+  const unsigned long long* g = packed(sm);
   unsigned long long t[PER];
   int mine = 0;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const bool live = slot_live(sm, i);
-    const unsigned long long K = live ? sm.cand[i * RT + threadIdx.x] : 0ull;
+  for (int j = 0; j < PER; ++j) {
+    const int i = j * RT + (int)threadIdx.x;
+    const unsigned long long K = i < n ? g[i] : 0ull;
     const int b = bin0(ckey_value(K), m);
-    t[i] = (live && b >= lo && b <= hi) ? K : 0ull;
-    mine += t[i] != 0ull ? 1 : 0;
+    t[j] = (i < n && b >= lo && b <= hi) ? K : 0ull;
+    mine += t[j] != 0ull ? 1 : 0;
   }
   long long tot;
   int o = (int)block_exscan<long long>((long long)mine, sm.red_l, tot);
-  // every slot is in registers now: the buffer is rewritten from the front
 #pragma unroll
-  for (int i = 0; i < PER; ++i)
-    if (t[i] != 0ull) {
-      if (o < SCAP) sm.cand[o] = t[i];
-      ++o;
-    }
+  for (int j = 0; j < PER; ++j)
+    if (t[j] != 0ull) sm.cand[o++] = t[j];
   __syncthreads();
-  return (int)min(tot, (long long)SCAP);
+  return (int)tot;
 }
 
-// Exact mass and count of the gathered candidates in bucket b, and (for
+// Exact mass and count of the n packed candidates in bucket b, and (for
 // min-p) of those with key >= kt, plus the smallest such key.
-__device__ __noinline__ void gathered_bucket_stats(RSmem& sm, float m, int b, uint32_t kt,
+__device__ __noinline__ void gathered_bucket_stats(RSmem& sm, int n, float m, int b, uint32_t kt,
                                                    double& mass, long long& cnt, double& kept_mass,
                                                    long long& kept_cnt, unsigned long long& k_min) {
-  constexpr int PER = CAP / RT;
+  const unsigned long long* g = packed(sm);
   double ms = 0.0, km = 0.0;
   long long c = 0, kc = 0;
   unsigned long long kmn = ~0ull;
-#pragma unroll 4
-  for (int i = 0; i < PER; ++i) {
-    const bool live = slot_live(sm, i);
-    const unsigned long long K = live ? sm.cand[i * RT + threadIdx.x] : 0ull;
+  for (int i = threadIdx.x; i < n; i += RT) {
+    const unsigned long long K = g[i];
     const float v = ckey_value(K);
-    const bool in = live && bin0(v, m) == b;
-    const double q = in ? qmass(sm, v, m) : 0.0;
-    const bool kept = in && (uint32_t)(K >> 32) >= kt;
+    if (bin0(v, m) != b) continue;
+    const double q = qmass(sm, v, m);
     ms += q;
-    c += in ? 1 : 0;
-    km += kept ? q : 0.0;
-    kc += kept ? 1 : 0;
-    kmn = (kept && K < kmn) ? K : kmn;
+    ++c;
+    if ((uint32_t)(K >> 32) >= kt) {
+      km += q;
+      ++kc;
+      kmn = K < kmn ? K : kmn;
+    }
   }
   double v[4] = {ms, (double)c, km, (double)kc};  // counts are exact in a double
   block_sum_multi<4>(v, sm);
@@ -1117,19 +1126,18 @@ __device__ __noinline__ void gathered_bucket_stats(RSmem& sm, float m, int b, ui
   k_min = block_ext_u<false>(kmn, sm);
 }
 
-// Exact masses and counts of the gathered candidates of buckets lo..hi
-// (hi - lo <= 2), in one sweep over the per-warp slices.
-__device__ __noinline__ void window_stats(RSmem& sm, float m, int lo, int hi, double (&wm)[3],
-                                          long long (&wc)[3]) {
-  constexpr int PER = CAP / RT;
+// Exact masses and counts of the n packed candidates of buckets lo..hi
+// (hi - lo <= 2).
+__device__ __noinline__ void window_stats(RSmem& sm, int n, float m, int lo, int hi,
+                                          double (&wm)[3], long long (&wc)[3]) {
+  const unsigned long long* g = packed(sm);
   double ms[3] = {0.0, 0.0, 0.0};
   long long c[3] = {0, 0, 0};
-#pragma unroll 4
-  for (int i = 0; i < PER; ++i) {
-    const bool live = slot_live(sm, i);
-    const float v = ckey_value(live ? sm.cand[i * RT + threadIdx.x] : 0ull);
-    const int w = live ? bin0(v, m) - lo : -1;
-    const double q = (w >= 0 && w <= hi - lo) ? qmass(sm, v, m) : 0.0;
+  for (int i = threadIdx.x; i < n; i += RT) {
+    const float v = ckey_value(g[i]);
+    const int w = bin0(v, m) - lo;
+    if (w < 0 || w > hi - lo) continue;
+    const double q = qmass(sm, v, m);
 #pragma unroll
     for (int u = 0; u < 3; ++u) {
       ms[u] += w == u ? q : 0.0;
@@ -1265,7 +1273,8 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
     pl.g_hi = bk;
     pass2<VEC>(sm, x, V, m, false, pl, P);
     if (P.overflow) return false;
-    const int n = compact_gathered(sm, m, 0, bk);
+    const int ng = pack_gathered(sm);
+    const int n = compact_gathered(sm, ng, m, 0, bk);
     sort_and_scan(sm, n, m);
     const int jk = min(k, n) - 1;
     Cut ck{sm.cand[jk], (long long)jk + 1, sm.cq[jk]};
@@ -1326,18 +1335,19 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
     if (gathered > SCAP) return false;  // keep the per-warp slices far from full
     pass2<VEC>(sm, x, V, m, p_on, pl, P);
     if (P.overflow) return false;
+    const int ng = pack_gathered(sm);
 
     bool have = false;
     if (mu_on) {
       double mass, kmass;
       long long cnt, kcnt;
       unsigned long long kmin;
-      gathered_bucket_stats(sm, m, bm, kt, mass, cnt, kmass, kcnt, kmin);
+      gathered_bucket_stats(sm, ng, m, bm, kt, mass, cnt, kmass, kcnt, kmin);
       if (kcnt == 0 && bprev >= 0) {
         // nothing of bucket bm is kept: the min-p prefix ends with bucket bprev
         double m2, k2;
         long long c2, kc2;
-        gathered_bucket_stats(sm, m, bprev, 0u, m2, c2, k2, kc2, kmin);
+        gathered_bucket_stats(sm, ng, m, bprev, 0u, m2, c2, k2, kc2, kmin);
       }
       best = Cut{kmin, before_mu + kcnt, P.a_mu + kmass};
       have = true;
@@ -1347,7 +1357,7 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
       // the crossing bucket, from the exact masses of the gathered window
       double wm[3];
       long long wc[3];
-      window_stats(sm, m, lo, hi, wm, wc);
+      window_stats(sm, ng, m, lo, hi, wm, wc);
       double before = P.a_p;
       long long cbefore = before_win;
       int c = -1;
@@ -1363,7 +1373,7 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
         if (narrowed) continue;
         return false;
       }
-      const int n = compact_gathered(sm, m, c, c);
+      const int n = compact_gathered(sm, ng, m, c, c);
       sort_and_scan(sm, n, m);
       const int jp = first_mass_hit(sm, 0, n, before, 0.0, kMassGE, target);
       const Cut cp{sm.cand[jp], cbefore + jp + 1, before + sm.cq[jp]};
