@@ -169,6 +169,65 @@ def test_filter_flat_rows_full_vocab(cuda_lib):
     assert not (mism & (gaps > 1e-12)).any(), np.flatnonzero(mism)
 
 
+def _estimate_defeating_rows():
+    """Rows whose logits sit on bucket edges, so that weighting every element
+    by its bucket's mid-point mass (the resolver's planning estimate) is off
+    by up to 0.39 % per bucket: the top-p crossing lands outside the planned
+    window (a retry with the wider window, or the exact search). The rows'
+    min-p alternates between off and 0.01."""
+    rng = np.random.Generator(np.random.PCG64(79))
+    V = 152064
+    rows, ps = [], []
+    # a heavy bucket at its top edge followed by one at its bottom edge: the
+    # crossing's bucket is misjudged by one. With 1300 logits per bucket the
+    # 3-bucket retry holds it; with 6000 the window exceeds the candidate
+    # buffer and the exact search decides.
+    for n, p_list in ((1300, (0.5026, 0.5032)), (6000, (0.5025,))):
+        s = np.full(V, -40.0, np.float32)
+        s[0] = 0.0
+        s[1:n + 1] = np.float32(-10 / 128)
+        s[n + 1:2 * n + 1] = np.float32(-12 / 128 + 2.0 ** -20)
+        s[2 * n + 1:2 * n + 8000] = (rng.standard_normal(7999) * 0.5 - 8).astype(np.float32)
+        for p in p_list:
+            rows.append(s)
+            ps.append(p)
+    # 600 light buckets of three equal logits, then 150,000 logits on one
+    # bucket edge: the mass estimate shifts the crossing by >10 buckets
+    s = np.empty(V, np.float32)
+    s[0] = 0.0
+    for b in range(1, 601):
+        s[3 * b - 2:3 * b + 1] = np.float32(-(b + 0.5) / 128)
+    s[1801:] = np.float32(-700 / 128)
+    for p in (0.3411794900894165, 0.36984652280807495):
+        rows.append(s)
+        ps.append(p)
+    S = np.stack(rows)
+    T = S.shape[0]
+    md = {
+        "top_k": np.zeros(T, np.int32),
+        "top_p": np.array(ps, np.float32),
+        "min_p": np.where(np.arange(T) % 2 == 1, 0.01, 0.0).astype(np.float32),
+        "temperature": np.ones(T, np.float32),
+        "target": np.zeros(T, np.int64),
+    }
+    return S, md
+
+
+def test_filter_when_the_planning_estimate_is_wrong(cuda_lib):
+    sts = cuda_lib
+    S, md = _estimate_defeating_rows()
+    out = sts.sts_filter_logits(torch.from_numpy(S).cuda(), torch.from_numpy(md["top_k"]).cuda(),
+                                torch.from_numpy(md["top_p"]).cuda(),
+                                torch.from_numpy(md["min_p"]).cuda(), check=True)
+    ref = oracle.filter_rows(S, md)
+    assert oracle.row_gaps(S, md).min() > 1e-6  # no near-tie decides these rows
+    T = S.shape[0]
+    size = out["size"].cpu().numpy()
+    cid = out["cut_id"].cpu().numpy()
+    assert np.array_equal(size, ref["size"]) and np.array_equal(cid, ref["cut_id"]), (size, ref["size"])
+    assert np.array_equal(out["cut_logit"].cpu().numpy(), S[np.arange(T), ref["cut_id"]])
+
+
 def test_filter_rejects_bad_rows(cuda_lib):
     sts = cuda_lib
     T, V = 4, 100
