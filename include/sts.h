@@ -83,8 +83,7 @@ typedef struct {
   int64_t T;           /* rows (scored tokens), >= 1 */
   int64_t d;           /* hidden size, >= 8, multiple of 8 */
   int64_t V;           /* vocabulary size, >= 1, < 2^31 */
-  int64_t vocab_chunk; /* backward vocab chunk (multiple of 256); 0: automatic
-                          (see sts_vocab_chunk) */
+  int64_t vocab_chunk; /* backward vocab chunk (multiple of 256); 0: 16384 */
   int64_t row_chunk;   /* forward row chunk (multiple of 128); 0: default */
 } sts_shape;
 
@@ -117,13 +116,11 @@ typedef struct {
  * 2 sts_filter_logits. Returns 0 for an invalid shape. */
 size_t sts_workspace_bytes(const sts_shape* shape, int pass);
 
-/* The vocabulary chunk the backward uses for this shape: shape->vocab_chunk
- * when set (clamped to V rounded up to 256), else the multiple of 256 in
- * [4096, 32768] that minimises a model of the three backward GEMMs' time
- * (waves of 148 persistent CTAs times each tile's contraction length, plus a
- * fixed cost per launch). A pure function of the shape, so workspace sizes
- * do not depend on the device. Returns -1 for an invalid shape. Not from the
- * pages: they chunk the vocabulary but fix no chunk size. */
+/* The vocabulary chunk the backward uses for this shape: shape->vocab_chunk,
+ * or 16384 when it is 0, clamped to V rounded up to 256. A pure function of
+ * the shape (workspace sizes do not depend on the device). Returns -1 for an
+ * invalid shape. Not from the pages: they chunk the vocabulary but fix no
+ * chunk size. */
 int64_t sts_vocab_chunk(const sts_shape* shape);
 
 /* Forward: logprob[T] (fp32) and the saved per-row scalars.

@@ -23,9 +23,7 @@
 namespace sts {
 namespace {
 
-constexpr int64_t kMinAutoVocabChunk = 4096;   // default backward vocabulary chunk: searched
-constexpr int64_t kMaxAutoVocabChunk = 32768;   // over multiples of 256 in this range
-constexpr int64_t kWaveCtas = 148;              // persistent GEMM CTAs (one per B200 SM)
+constexpr int64_t kDefaultVocabChunk = 16384;
 constexpr size_t kDefaultChunkBytes = size_t(4) << 30;  // forward logits chunk budget
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -196,39 +194,9 @@ int64_t row_chunk(const sts_shape* s) {
   return rc < Tpad ? rc : Tpad;
 }
 
-// Modelled time of the three backward GEMMs for vocabulary chunk Vc, in
-// K-steps per SM: every launch runs ceil(tiles / 148) waves of tiles whose
-// length is the contraction (d for dZ, T for dW, the chunk width for dH),
-// plus a fixed cost per launch for pipeline fill and drain. Wave quantisation
-// makes any single fixed chunk a poor choice for some shapes.
-int64_t backward_cost(int64_t T, int64_t d, int64_t V, int64_t Vc) {
-  auto waves = [](int64_t tiles) { return (tiles + kWaveCtas - 1) / kWaveCtas; };
-  const int64_t tm = (T + GEMM_BM - 1) / GEMM_BM, dn = (d + GEMM_BN - 1) / GEMM_BN;
-  const int64_t kLaunch = 2048;
-  int64_t c = 0;
-  for (int64_t v0 = 0; v0 < V; v0 += Vc) {
-    const int64_t w = std::min(Vc, V - v0);
-    c += waves(tm * ((w + GEMM_BN - 1) / GEMM_BN)) * d;  // dZ: T x w tiles, K = d
-    c += waves(((w + GEMM_BM - 1) / GEMM_BM) * dn) * T;  // dW: w x d tiles, K = T
-    c += waves(tm * dn) * w;                              // dH: T x d tiles, K = w
-    c += 3 * kLaunch;
-  }
-  return c;
-}
-
 int64_t vocab_chunk(const sts_shape* s) {
   const int64_t Vpad = (s->V + 255) / 256 * 256;
-  int64_t vc = s->vocab_chunk;
-  if (vc == 0) {
-    int64_t best = -1;
-    for (int64_t c = kMinAutoVocabChunk; c <= kMaxAutoVocabChunk; c += 256) {
-      const int64_t cost = backward_cost(s->T, s->d, s->V, c);
-      if (best < 0 || cost < best) {
-        best = cost;
-        vc = c;
-      }
-    }
-  }
+  const int64_t vc = s->vocab_chunk ? s->vocab_chunk : kDefaultVocabChunk;
   return vc < Vpad ? vc : Vpad;
 }
 

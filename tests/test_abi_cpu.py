@@ -51,9 +51,8 @@ def test_workspace_sizes(lib):
     flt = lib.sts_workspace_bytes(ctypes.byref(sh), 2)
     # forward: header + flags + one row chunk of fp32 logits (row stride padded to 4)
     assert fwd >= 1024 * 50000 * 4 and fwd % 1024 == 0
-    # backward: one vocab chunk (the automatic choice) of bf16 dZ for all rows
-    vc = lib.sts_vocab_chunk(ctypes.byref(sh))
-    assert vc >= 4096 and bwd >= 1000 * vc * 2
+    # backward: one vocab chunk (default 16384 columns) of bf16 dZ for all rows
+    assert lib.sts_vocab_chunk(ctypes.byref(sh)) == 16384 and bwd >= 1000 * 16384 * 2
     assert flt >= 1000 * 4
     sh2 = _shape(T=1000, d=128, V=50000, vc=8192, rc=256)
     assert lib.sts_workspace_bytes(ctypes.byref(sh2), 1) < bwd
@@ -146,30 +145,13 @@ def test_binding_rejects_wrong_metadata_length():
         sts._rows(5, None, t, k, t, t)
 
 
-def _backward_cost_model(T, d, V, Vc, ctas=148, launch=2048):
-    """The documented model, restated: waves of ``ctas`` tiles times each
-    tile's contraction length, plus a fixed cost per launch."""
-    waves = lambda tiles: -(-tiles // ctas)
-    tm, dn = -(-T // 128), -(-d // 256)
-    c = 0
-    for v0 in range(0, V, Vc):
-        w = min(Vc, V - v0)
-        c += waves(tm * -(-w // 256)) * d + waves(-(-w // 128) * dn) * T + waves(tm * dn) * w + 3 * launch
-    return c
-
-
 def test_vocab_chunk_choice():
     for T, d, V in [(16384, 5120, 152064), (8192, 4096, 151936), (32768, 4096, 262144),
                     (4096, 2048, 32768), (300, 64, 100000)]:
         vc = sts.sts_vocab_chunk(T, d, V)
-        assert vc % 256 == 0 and 4096 <= vc <= 32768
-        costs = {c: _backward_cost_model(T, d, V, c) for c in range(4096, 32769, 256)}
-        assert costs[vc] == min(costs.values())
-        assert vc == min(c for c in costs if costs[c] == costs[vc])  # first minimum
-        # an explicit chunk is kept; any chunk is clamped to V rounded up to 256
-        assert sts.sts_vocab_chunk(T, d, V, vocab_chunk=8192) == 8192
-        # the workspace follows the chosen chunk
-        assert sts.sts_workspace_bytes(T, d, V, 1) >= T * vc * 2
+        assert vc == min(16384, (V + 255) // 256 * 256)
+        assert sts.sts_vocab_chunk(T, d, V, vocab_chunk=8192) == 8192  # an explicit chunk is kept
+        assert sts.sts_workspace_bytes(T, d, V, 1) >= T * vc * 2  # the workspace follows it
     assert sts.sts_vocab_chunk(64, 128, 1000) == 1024
     assert sts.sts_vocab_chunk(64, 128, 1000, vocab_chunk=8192) == 1024
     with pytest.raises(sts.StsError):
