@@ -347,3 +347,48 @@ def row_gaps(s, rows):
         if mu > 0.0:
             out[t, 2] = float(np.min(np.abs(ss - f.m - math.log(mu))))
     return out
+
+
+# ---------------------------------------------------------------- policy-gradient coefficient
+
+def policy_grad(logprob, old_logprob, advantage, objective="cispo", eps_low=0.2, eps_high=0.2,
+                scale=1.0):
+    """Upstream gradient g_t = dL/dlogprob_t of a policy-gradient token loss,
+    to be fed to the backward as grad_logprob.
+
+    [align-v2] section 5.4 A, "Why the in-chunk form works for this loss": the
+    per-token logit gradient of the objective J is c_t (softmax - onehot) with a
+    token coefficient known from the fresh logprob; the loss the optimiser
+    minimises is L = -J. With r_t = exp(logprob_t - old_logprob_t):
+
+    * "cispo" (CISPO, cited there as arXiv:2506.13585 Sec. 3.1 Eq. 4-5): J =
+      sum_t sg(min(r_t, 1 + eps_high)) A_t logprob_t, the importance weight a
+      stop-gradient constant with no lower bound, so
+      g_t = -scale * A_t * min(r_t, 1 + eps_high).
+    * "clipped" (the clipped surrogate of the same passage): J = sum_t
+      min(r_t A_t, clip(r_t, 1 - eps_low, 1 + eps_high) A_t); where the clip
+      binds the term is constant in logprob, elsewhere d(r_t A_t)/dlogprob_t =
+      r_t A_t, so g_t = -scale * A_t * r_t * 1[not clipped], clipped meaning
+      r_t > 1 + eps_high for A_t >= 0 and r_t < 1 - eps_low for A_t < 0.
+
+    ``scale`` carries the loss normalisation (for example 1 / tokens). Rows
+    whose logprob is -inf (replayed token outside the support) or NaN (an
+    invalid row) get g_t = 0. Float64 throughout.
+    """
+    lp = np.asarray(logprob, dtype=np.float64)
+    old = np.asarray(old_logprob, dtype=np.float64)
+    adv = np.asarray(advantage, dtype=np.float64)
+    out = np.zeros(lp.shape, dtype=np.float64)
+    for t in range(lp.shape[0]):
+        if not np.isfinite(lp[t]):
+            continue
+        r = math.exp(lp[t] - old[t])
+        if objective == "cispo":
+            out[t] = -scale * adv[t] * min(r, 1.0 + eps_high)
+        elif objective == "clipped":
+            clipped = r > 1.0 + eps_high if adv[t] >= 0 else r < 1.0 - eps_low
+            out[t] = 0.0 if clipped else -scale * adv[t] * r
+        else:
+            raise ValueError(f"unknown objective {objective!r}")
+    return out
+

@@ -403,3 +403,56 @@ def test_stress_workload_duplicates_rows():
     d = workloads.make(5, T=8, with_weights=False)
     assert len(d["dup_dst"]) == round(0.05 * 262144)
     assert (d["dup_src"] < d["dup_dst"]).all()
+
+
+# ---------------------------------------------------------------- policy-gradient coefficient
+
+def _pg_inputs(n=400, seed=31):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    lp = -rng.exponential(2.0, n)
+    old = lp + rng.normal(0.0, 0.4, n)  # ratios spread around 1, many clipped
+    adv = rng.normal(0.0, 1.0, n)
+    adv[::17] = 0.0
+    return lp, old, adv
+
+
+@pytest.mark.parametrize("objective", ["cispo", "clipped"])
+def test_policy_grad_is_the_autograd_of_the_loss(objective):
+    """The coefficient is the float64 autograd of the loss written out as the
+    passage defines it: L = -sum sg(min(r, 1+eh)) A logprob (CISPO) or
+    L = -sum min(r A, clip(r, 1-el, 1+eh) A) (clipped surrogate)."""
+    lp, old, adv = _pg_inputs()
+    el, eh, scale = 0.2, 0.28, 1.0 / 400
+    x = torch.tensor(lp, dtype=torch.float64, requires_grad=True)
+    o = torch.tensor(old, dtype=torch.float64)
+    a = torch.tensor(adv, dtype=torch.float64)
+    r = torch.exp(x - o)
+    if objective == "cispo":
+        loss = -(torch.clamp(r, max=1 + eh).detach() * a * x).sum() * scale
+    else:
+        loss = -torch.minimum(r * a, torch.clamp(r, 1 - el, 1 + eh) * a).sum() * scale
+    loss.backward()
+    got = oracle.policy_grad(lp, old, adv, objective, el, eh, scale)
+    rr = np.exp(lp - old)
+    # away from the clip boundaries, where the loss is not differentiable
+    ok = (np.abs(rr - (1 + eh)) > 1e-9) & (np.abs(rr - (1 - el)) > 1e-9)
+    assert ok.sum() > 350
+    np.testing.assert_allclose(got[ok], x.grad.numpy()[ok], rtol=1e-12, atol=1e-15)
+    # both clip regimes occur in the sample
+    assert (rr > 1 + eh).any() and (rr < 1 - el).any()
+
+
+def test_policy_grad_special_rows():
+    lp = np.array([-np.inf, np.nan, -1.0, -1.0, -1.0, -1.0])
+    old = np.array([-2.0, -2.0, -1.0, -1.5, -0.5, -1.5])
+    adv = np.array([1.0, 1.0, 0.0, 2.0, -2.0, -2.0])
+    c = oracle.policy_grad(lp, old, adv, "cispo", 0.2, 0.3, 1.0)
+    assert c[0] == 0.0 and c[1] == 0.0 and c[2] == 0.0  # out of support, invalid, A = 0
+    assert c[3] == -2.0 * 1.3  # r = e^0.5 > 1.3: the weight saturates at 1 + eps_high
+    assert c[4] == pytest.approx(2.0 * np.exp(-0.5), rel=1e-15)  # no lower bound for CISPO
+    k = oracle.policy_grad(lp, old, adv, "clipped", 0.2, 0.3, 1.0)
+    assert k[3] == 0.0  # A > 0, r above 1 + eps_high: clipped
+    assert k[4] == 0.0  # A < 0, r = e^-0.5 below 1 - eps_low: clipped
+    assert k[5] == pytest.approx(2.0 * np.exp(0.5), rel=1e-15)  # A < 0, r above 1: not clipped
+    with pytest.raises(ValueError):
+        oracle.policy_grad(lp, old, adv, "ppo")
