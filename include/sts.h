@@ -199,6 +199,27 @@ sts_status sts_probe_mass_exp(const float* s, float m, double* mass, double* lib
  * ws. first_bad_row (may be NULL) receives the lowest failing row or -1. */
 sts_status sts_get_status(const void* ws, sts_stream_t stream, int64_t* first_bad_row);
 
+/* Policy-gradient objectives for sts_policy_grad. */
+typedef enum { STS_PG_CISPO = 0, STS_PG_CLIPPED = 1 } sts_pg_objective;
+
+/* The upstream gradient grad_logprob[t] = dL/dlogprob_t of a policy-gradient
+ * token loss L = -J, formed from the forward's fresh logprobs and passed to
+ * sts_backward ("align architecture v2: proposal", section 5.4 A, "Why the
+ * in-chunk form works for this loss": the logit gradient is a per-token
+ * coefficient times (softmax - onehot)). With r_t = exp(logprob_t -
+ * old_logprob_t), in float64:
+ *   STS_PG_CISPO    -scale * A_t * min(r_t, 1 + eps_high)   (weight held constant)
+ *   STS_PG_CLIPPED  -scale * A_t * r_t, 0 where the clip binds: r_t > 1 + eps_high
+ *                   with A_t >= 0, r_t < 1 - eps_low with A_t < 0
+ * Rows whose logprob is not finite (-inf out of support, NaN invalid) get 0.
+ * All arrays [T] fp32 on the device; scale carries the loss normalisation.
+ * Returns STS_ERR_SHAPE for T < 0, an unknown objective, negative or
+ * non-finite eps or a non-finite scale; STS_ERR_NULL for a NULL array (T > 0).
+ * Asynchronous on stream; allocates nothing. */
+sts_status sts_policy_grad(int64_t T, const float* logprob, const float* old_logprob,
+                           const float* advantage, int objective, float eps_low, float eps_high,
+                           float scale, float* grad_logprob, sts_stream_t stream);
+
 const char* sts_status_string(sts_status status);
 
 /* Kernel kinds for the launch counters and the timing facility below. */

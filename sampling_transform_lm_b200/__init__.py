@@ -32,6 +32,7 @@ __all__ = [
     "sts_sample",
     "sts_filter_logits",
     "sts_scaled_logits",
+    "sts_policy_grad",
     "sts_get_status",
     "sts_status_string",
     "sts_probe_mass_exp",
@@ -76,6 +77,7 @@ EXPORTED_SYMBOLS = (
     "sts_timing_enable",
     "sts_timing_read",
     "sts_filter_logits_noalloc",
+    "sts_policy_grad",
 )
 
 
@@ -143,6 +145,9 @@ def load():
     lib.sts_status_string.restype = ctypes.c_char_p
     lib.sts_probe_mass_exp.argtypes = [P, ctypes.c_float, P, P, I64, P]
     lib.sts_probe_mass_exp.restype = ctypes.c_int
+    lib.sts_policy_grad.argtypes = [I64, P, P, P, ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                    ctypes.c_float, P, P]
+    lib.sts_policy_grad.restype = ctypes.c_int
     lib.sts_launch_count.argtypes = [ctypes.c_int]
     lib.sts_launch_count.restype = ctypes.c_int64
     lib.sts_timing_enable.argtypes = [ctypes.c_int]
@@ -376,6 +381,31 @@ def sts_filter_logits_noalloc(S, top_k, top_p, min_p, *, support_size, cut_logit
     _check(lib.sts_filter_logits_noalloc(ctypes.byref(sh), _ptr(S), ctypes.byref(rows),
                                          _ptr(support_size), _ptr(cut_logit), _ptr(cut_id),
                                          _ptr(mask), _stream(stream)), "sts_filter_logits_noalloc")
+
+
+PG_OBJECTIVES = {"cispo": 0, "clipped": 1}
+
+
+def sts_policy_grad(logprob, old_logprob, advantage, *, objective="cispo", eps_low=0.2,
+                    eps_high=0.2, scale=1.0, out=None, stream=None):
+    """grad_logprob [T] (fp32) of a policy-gradient token loss from the fresh
+    logprobs, to pass to sts_backward: CISPO (-scale A min(r, 1 + eps_high))
+    or the clipped surrogate (-scale A r where the clip does not bind)."""
+    lib = load()
+    if objective not in PG_OBJECTIVES:
+        raise StsError(STS_ERR_SHAPE, f"objective must be one of {sorted(PG_OBJECTIVES)}")
+    T = logprob.shape[0]
+    for name, t in (("logprob", logprob), ("old_logprob", old_logprob), ("advantage", advantage)):
+        _need(t, torch.float32, name, (T,))
+    if out is None:
+        out = torch.empty(T, dtype=torch.float32, device=logprob.device)
+    _need(out, torch.float32, "out", (T,))
+    st = lib.sts_policy_grad(int(T), _ptr(logprob), _ptr(old_logprob), _ptr(advantage),
+                             PG_OBJECTIVES[objective], float(eps_low), float(eps_high), float(scale),
+                             _ptr(out), _stream(stream))
+    if st != STS_OK:
+        raise StsError(st, "sts_policy_grad")
+    return out
 
 
 def sts_scaled_logits(H, W, temperature, t0=0, rows=None, v0=0, cols=None, *, out=None,

@@ -156,3 +156,15 @@ def test_vocab_chunk_choice():
     assert sts.sts_vocab_chunk(64, 128, 1000, vocab_chunk=8192) == 1024
     with pytest.raises(sts.StsError):
         sts.sts_vocab_chunk(64, 128, 1000, vocab_chunk=100)  # not a multiple of 256
+
+
+def test_policy_grad_host_checks(lib):
+    """Argument errors return before any device work (no GPU needed)."""
+    null = ctypes.c_void_p(0)
+    assert lib.sts_policy_grad(-1, null, null, null, 0, 0.2, 0.2, 1.0, null, null) == 2
+    assert lib.sts_policy_grad(4, null, null, null, 7, 0.2, 0.2, 1.0, null, null) == 2
+    assert lib.sts_policy_grad(4, null, null, null, 0, -0.1, 0.2, 1.0, null, null) == 2
+    assert lib.sts_policy_grad(4, null, null, null, 1, 0.2, float("nan"), 1.0, null, null) == 2
+    assert lib.sts_policy_grad(4, null, null, null, 0, 0.2, 0.2, float("inf"), null, null) == 2
+    assert lib.sts_policy_grad(4, null, null, null, 0, 0.2, 0.2, 1.0, null, null) == 1
+    assert lib.sts_policy_grad(0, null, null, null, 1, 0.2, 0.2, 1.0, null, null) == 0

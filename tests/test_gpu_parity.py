@@ -246,3 +246,57 @@ def test_workload2_forward_all_rows(cuda_lib):
     _check_forward(out, s, rows, ref)
     flagged = near_gap_rows(s, rows)
     print(f"workload 2: {int(flagged.sum())} near-gap rows of {len(flagged)}")
+
+
+@pytest.mark.parametrize("objective", ["cispo", "clipped"])
+def test_policy_grad_matches_oracle(cuda_lib, objective):
+    """The policy-gradient coefficient, elementwise against the oracle."""
+    sts = cuda_lib
+    rng = np.random.Generator(np.random.PCG64(40))
+    T = 5003  # several blocks and a ragged tail
+    lp = (-rng.exponential(2.0, T)).astype(np.float32)
+    old = (lp + rng.normal(0.0, 0.4, T)).astype(np.float32)
+    adv = rng.normal(0.0, 1.0, T).astype(np.float32)
+    lp[::97] = -np.inf  # replayed token outside the support
+    lp[5::211] = np.nan  # invalid rows
+    adv[::13] = 0.0
+    cu = lambda a: torch.from_numpy(a).cuda()
+    got = sts.sts_policy_grad(cu(lp), cu(old), cu(adv), objective=objective, eps_low=0.2,
+                              eps_high=0.28, scale=1.0 / T).cpu().numpy()
+    ref = oracle.policy_grad(lp, old, adv, objective, np.float32(0.2), np.float32(0.28),
+                             np.float32(1.0 / T))
+    rr = np.exp(lp.astype(np.float64) - old)
+    near = (np.abs(rr - (1 + np.float32(0.28))) < 1e-12) | (np.abs(rr - (1 - np.float32(0.2))) < 1e-12)
+    assert not near.any()  # no clip decision rests on rounding
+    np.testing.assert_allclose(got, ref, rtol=2e-7, atol=1e-30)
+    assert (got[::97] == 0).all() and (got[5::211] == 0).all()
+    with pytest.raises(sts.StsError):
+        sts.sts_policy_grad(cu(lp), cu(old), cu(adv), objective="ppo")
+
+
+def test_policy_gradient_through_the_backward(cuda_lib):
+    """CISPO end to end on the tiny workload: the coefficient formed from the
+    GPU's fresh logprobs drives the backward; dH and dW match the oracle's
+    backward driven by the oracle's coefficient from its own logprobs."""
+    data = workloads.make(1)
+    meta = {k: data[k] for k in ("temperature", "top_k", "top_p", "min_p")}
+    Hf, Wf, s, rows = _oracle_case(data["H"], data["W"], meta, data["u"])
+    ref = oracle.forward(Hf, Wf, rows, s=s)
+    rng = np.random.Generator(np.random.PCG64(41))
+    T = len(rows["target"])
+    old = (np.where(np.isfinite(ref["logprob"]), ref["logprob"], -5.0) + rng.normal(0, 0.3, T))
+    old = old.astype(np.float32)
+    adv = rng.normal(0.0, 1.0, T).astype(np.float32)
+    fwd = _run(cuda_lib, data["H"], data["W"], rows)
+    same = _check_forward(fwd, s, rows, ref)
+    lp_gpu = torch.from_numpy(fwd["logprob"]).cuda()
+    g = cuda_lib.sts_policy_grad(lp_gpu, torch.from_numpy(old).cuda(), torch.from_numpy(adv).cuda(),
+                                 objective="cispo", eps_high=0.28, scale=1.0 / T).cpu().numpy()
+    g_ref = oracle.policy_grad(ref["logprob"], old, adv, "cispo", 0.2, np.float32(0.28),
+                               np.float32(1.0 / T))
+    assert np.abs(g - g_ref)[same].max() <= 1e-2 * np.abs(g_ref).max()
+    gm = np.where(same, g, 0.0).astype(np.float32)
+    out = _run(cuda_lib, data["H"], data["W"], rows, grad=gm)
+    dH, dW = oracle.backward(Hf, Wf, rows, np.where(same, g_ref, 0.0), s=s)
+    assert rel_fro(out["dH"], dH) < GRAD_RTOL
+    assert rel_fro(out["dW"], dW) < GRAD_RTOL
