@@ -63,6 +63,15 @@ _TRAFFIC_SOURCES = {
 }
 
 
+def source_code_only(text):
+    """The source with comments and blank lines removed, so that a change to
+    comments alone does not invalidate a recorded measurement."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def recorded_traffic(T, d, V, kernel):
     """DRAM bytes (read + write) per launch of ``kernel`` from the committed
     ncu capture of this workload (profiles/dram_traffic_T*_d*_V*.json), or
@@ -76,8 +85,8 @@ def recorded_traffic(T, d, V, kernel):
     group = "resolve" if kernel == "resolve" else "gemm"
     h = hashlib.sha256()
     for name in _TRAFFIC_SOURCES[group]:
-        with open(os.path.join(ROOT, "sampling_transform_lm_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "sampling_transform_lm_b200", "csrc", name)) as f:
+            h.update(source_code_only(f.read()).encode())
     k = rec.get("kernels", {}).get(kernel)
     if k is None or rec.get("sources", {}).get(group) != h.hexdigest()[:16]:
         return None

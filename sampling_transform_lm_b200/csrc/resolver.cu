@@ -28,13 +28,16 @@
 //                monotone in s, so every bucket is a contiguous run of the
 //                order.
 //   planning     from the counts alone: the top-k cut's bucket; the top-p
-//                crossing's bucket estimated with mid-bucket weights, widened
-//                to a 3-bucket window; the min-p threshold's bucket and the
-//                non-empty bucket before it.
-//   exact pass   (from L2) float64 masses of every element, summed in
-//                registers (the total, the mass before the window, the mass
-//                before the min-p bucket), and the elements of the planned
-//                buckets gathered into per-warp slices of a candidate buffer.
+//                crossing's bucket estimated with mid-bucket weights (with a
+//                neighbour where the estimate lies within six sigma of an
+//                edge; one retry with a 3-bucket window if the exact masses
+//                then place the crossing outside); the min-p threshold's
+//                bucket and the non-empty bucket before it.
+//   exact pass   (from L2: the count pass marks the row's lines evict-last)
+//                float64 masses of every element, summed in registers (the
+//                total, the mass before the window, the mass before the min-p
+//                bucket), and the elements of the planned buckets gathered
+//                into per-warp slices of a candidate buffer, then packed.
 //   finish       exact masses of the window buckets place the crossing in one
 //                bucket; its elements are sorted by composite key (a bitonic
 //                network held mostly in registers and warp shuffles) and

@@ -52,6 +52,13 @@ def test_recorded_traffic_follows_the_kernel_sources(monkeypatch):
     assert bench.recorded_traffic(16384, 5120, 152064, "dw_gemm") is None
 
 
+def test_source_digest_ignores_comments():
+    code = "int a = 1;  // one\n\n/* block\n comment */int b = 2;\n"
+    assert bench.source_code_only(code) == "int a = 1;\nint b = 2;"
+    assert bench.source_code_only(code.replace("one", "uno")) == bench.source_code_only(code)
+    assert bench.source_code_only(code.replace("= 2", "= 3")) != bench.source_code_only(code)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
