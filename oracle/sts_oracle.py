@@ -27,7 +27,9 @@ Sources (cited by page title and section):
 * [align-v2] "align architecture v2: proposal", section 5.4 A "Fused head +
   policy-gradient token loss": the head needs fp32 *logits* from bf16
   operands, and the logit gradient of a selected-token logprob is
-  (onehot - softmax) scaled per token.
+  (onehot - softmax) scaled per token; "Why the in-chunk form works for this
+  loss" gives that per-token coefficient for CISPO and the clipped surrogate
+  (``policy_grad``).
 
 Readings taken where the pages are silent (each is a deliberate choice):
 
