@@ -273,7 +273,7 @@ def logit_grad(s, rows, grad_logprob):
     return dZ
 
 
-def backward(H, W, rows, grad_logprob, s=None, vocab_rows=None, vocab_slice=None):
+def backward(H, W, rows, grad_logprob, s=None, vocab_rows=None, vocab_slice=None, dZ=None):
     """Closed-form VJP: dH = dZ . W and dW = dZ^T . H in float64.
 
     [xorl#74] item 2 (recompute closed-form VJP) and "Acceptance criteria"
@@ -281,11 +281,14 @@ def backward(H, W, rows, grad_logprob, s=None, vocab_rows=None, vocab_slice=None
     vocabulary rows (the full [V, d] float64 matrix of the large workloads
     does not fit comfortably in host memory); ``vocab_slice`` widens W to
     float64 that many rows at a time for dH = sum over vocabulary slices.
+    ``dZ`` may pass the logit gradient already formed by ``logit_grad`` on the
+    same rows (for example row slice by row slice, in parallel).
     """
     H = np.asarray(H, dtype=np.float64)
-    if s is None:
-        s = scaled_logits(H, W, rows["temperature"], vocab_slice=vocab_slice)
-    dZ = logit_grad(s, rows, grad_logprob)
+    if dZ is None:
+        if s is None:
+            s = scaled_logits(H, W, rows["temperature"], vocab_slice=vocab_slice)
+        dZ = logit_grad(s, rows, grad_logprob)
     V = W.shape[0]
     step = V if vocab_slice is None else int(vocab_slice)
     dH = np.zeros((H.shape[0], H.shape[1]), dtype=np.float64)
@@ -321,13 +324,26 @@ def sample_rows(s, rows, u):
 
 
 def row_gaps(s, rows):
-    """Distance of each active threshold from its decision boundary.
+    """Distance of each threshold that can move the support from its decision
+    boundary, per row: columns (gap_k, gap_p, gap_mu).
 
     gap_k: s_(k-1) - s_(k) in scaled-logit units (exact ties report +inf: they
     are decided by token id, not by rounding). gap_p: min(p Z_k - C_(m_p - 1),
-    C_(m_p) - p Z_k) / Z_k. gap_mu: min_i |s_i - m - ln(min_p)|. Inactive rules
-    report +inf. A row whose smallest gap is tiny can legitimately resolve
-    differently under float32 logits or another summation order.
+    C_(m_p) - p Z_k) / Z_k, C the exclusive running mass (the first term only
+    when m_p > 1, the second only when m_p < k_eff: the first position is
+    always kept and a crossing cannot pass the last top-k position; +inf when
+    neither boundary exists). gap_mu: the distance in logit units of the min-p
+    threshold t = m + ln(min_p) from the last kept logit (unless that one ties
+    the row max, which min_p <= 1 always keeps) and from the first dropped one.
+
+    A rule reports its gap only where it can move the result: its prefix
+    length is within one position of the support size (m_r <= size + 1; the
+    support is the shortest of the prefixes, so crossing one boundary moves
+    m_r by one and can change the support only then). Rules that are off, or
+    whose prefix ends two or more positions after the support's, report +inf.
+    A row whose smallest gap is tiny can legitimately resolve differently
+    under float32 logits or another summation order ([xorl#74] item 1 fixes
+    the program; this measure only sorts rows for reporting).
     """
     s = np.asarray(s, dtype=np.float64)
     T, V = s.shape
@@ -336,18 +352,26 @@ def row_gaps(s, rows):
         k, p, mu = _row_meta(rows, t)
         f = filter_row(s[t], k, p, mu)
         ss = s[t, f.order]
-        if f.k_eff < V:
+        live = f.size + 1
+        if f.k_eff < V and f.k_eff <= live:
             g = ss[f.k_eff - 1] - ss[f.k_eff]
             out[t, 0] = g if g > 0 else np.inf
-        if p < 1.0:
+        if p < 1.0 and f.m_p <= live:
             q = np.exp(ss[: f.k_eff] - f.m)
             C = np.concatenate(([0.0], np.cumsum(q)))
             target = p * f.Z_k
-            lo = target - C[f.m_p - 1]
-            hi = C[f.m_p] - target
+            # no boundary below when only the first position is kept (C_0 = 0 <
+            # p Z_k for every p > 0), none above when every top-k position is
+            lo = target - C[f.m_p - 1] if f.m_p > 1 else np.inf
+            hi = C[f.m_p] - target if f.m_p < f.k_eff else np.inf
             out[t, 1] = min(lo, hi) / f.Z_k
-        if mu > 0.0:
-            out[t, 2] = float(np.min(np.abs(ss - f.m - math.log(mu))))
+        if mu > 0.0 and f.m_mu <= live:
+            thr = f.m + math.log(mu)
+            # the last kept logit bounds it from above unless it ties the max
+            # (min_p <= 1 always keeps the max); the first dropped one from below
+            up = ss[f.m_mu - 1] - thr if ss[f.m_mu - 1] < f.m else np.inf
+            down = thr - ss[f.m_mu] if f.m_mu < V else np.inf
+            out[t, 2] = min(up, down)
     return out
 
 
@@ -375,16 +399,25 @@ def policy_grad(logprob, old_logprob, advantage, objective="cispo", eps_low=0.2,
 
     ``scale`` carries the loss normalisation (for example 1 / tokens). Rows
     whose logprob is -inf (replayed token outside the support) or NaN (an
-    invalid row) get g_t = 0. Float64 throughout.
+    invalid row), or whose old logprob or advantage is not finite, get
+    g_t = 0; so do rows with scale * A_t == 0 (no signal). The ratio r_t is
+    +inf where exp overflows (logprob - old_logprob above ~709.8): the CISPO
+    weight is then 1 + eps_high, the clipped surrogate is clipped for A_t >= 0
+    and its gradient is infinite for A_t < 0. Float64 throughout.
     """
     lp = np.asarray(logprob, dtype=np.float64)
     old = np.asarray(old_logprob, dtype=np.float64)
     adv = np.asarray(advantage, dtype=np.float64)
     out = np.zeros(lp.shape, dtype=np.float64)
     for t in range(lp.shape[0]):
-        if not np.isfinite(lp[t]):
+        if not (np.isfinite(lp[t]) and np.isfinite(old[t]) and np.isfinite(adv[t])):
             continue
-        r = math.exp(lp[t] - old[t])
+        if scale * adv[t] == 0.0:
+            continue
+        try:
+            r = math.exp(lp[t] - old[t])
+        except OverflowError:
+            r = math.inf
         if objective == "cispo":
             out[t] = -scale * adv[t] * min(r, 1.0 + eps_high)
         elif objective == "clipped":

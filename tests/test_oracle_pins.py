@@ -384,6 +384,87 @@ def test_row_gaps_detect_near_ties():
     assert oracle.row_gaps(s, rows)[0, 0] == pytest.approx(1.0)
 
 
+GAPS = os.path.join(os.path.dirname(__file__), "golden", "threshold_gaps.json")
+
+
+def _gap_cases():
+    with open(GAPS) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _gap_cases(), ids=lambda c: c["name"])
+def test_row_gaps_hand_worked(case):
+    """gap_k, gap_p and gap_mu of hand-worked rows, including the rule that a
+    gap only counts where its prefix ends within one position of the support."""
+    s = np.log(np.array([case["weights"]], dtype=np.float64))
+    rows = _rows(1, 0, 1.0, case["top_k"], case["top_p"], case["min_p"])
+    assert oracle.filter_rows(s, rows)["size"][0] == case["size"]
+    got = oracle.row_gaps(s, rows)[0]
+    for g, want in zip(got, case["gaps"]):
+        if want == "inf":
+            assert g == math.inf
+        else:
+            assert abs(g - want) < 1e-12, (g, want)
+
+
+def _distance_to_change(f, x0, lo, hi):
+    """Distance from x0 to the nearest x in [lo, hi] where the integer
+    function f changes value, by bisection on each side (inf if none)."""
+    v0 = f(x0)
+    best = math.inf
+    for end in (lo, hi):
+        if f(end) == v0:
+            continue
+        a, b = x0, end  # f(a) == v0, f(b) != v0
+        for _ in range(200):
+            mid = 0.5 * (a + b)
+            if mid == a or mid == b:
+                break
+            if f(mid) == v0:
+                a = mid
+            else:
+                b = mid
+        best = min(best, abs(b - x0))
+    return best
+
+
+def test_row_gaps_match_bisection_on_random_rows():
+    """An independent formulation of the gaps on random rows (V <= 12): the
+    distance, found by bisection, by which p (in units of the top-k mass) or
+    ln(min_p) (in logit units) must move before the rule's own prefix length
+    m_p or m_mu changes -- compared with the closed forms of row_gaps wherever
+    the rule can move the support (its prefix within one position of it)."""
+    rng = np.random.default_rng(11)
+    checked = {"p": 0, "mu": 0}
+    for _ in range(400):
+        V = int(rng.integers(3, 12))
+        s = rng.standard_normal(V) * 2
+        k = int(rng.choice([0, 2, 3, V]))
+        p = float(np.float32(rng.choice([1.0, 0.5, 0.75, 0.9, 0.3])))
+        mu = float(np.float32(rng.choice([0.0, 0.1, 0.3, 0.6])))
+        rows = _rows(1, 0, 1.0, k, p, mu)
+        base = oracle.filter_row(s, k, p, mu)
+        gaps = oracle.row_gaps(s[None, :], rows)[0]
+        live = base.size + 1
+        if p < 1.0:
+            want = _distance_to_change(lambda x: oracle.filter_row(s, k, x, mu).m_p, p, 1e-12, 1.0 - 1e-15)
+            if base.m_p <= live:
+                assert abs(gaps[1] - want) < 1e-9, (gaps, want, s, k, p, mu)
+                checked["p"] += 1
+            else:
+                assert gaps[1] == math.inf
+        if mu > 0.0:
+            lm = math.log(mu)
+            want = _distance_to_change(
+                lambda x: oracle.filter_row(s, k, p, math.exp(x)).m_mu, lm, lm - 60.0, 0.0)
+            if base.m_mu <= live:
+                assert abs(gaps[2] - want) < 1e-9, (gaps, want, s, k, p, mu)
+                checked["mu"] += 1
+            else:
+                assert gaps[2] == math.inf
+    assert checked["p"] > 50 and checked["mu"] > 50, checked
+
+
 def test_workload_inputs_are_bf16_and_seeded():
     a = workloads.make(1)
     b = workloads.make(1)
@@ -456,3 +537,21 @@ def test_policy_grad_special_rows():
     assert k[5] == pytest.approx(2.0 * np.exp(0.5), rel=1e-15)  # A < 0, r above 1: not clipped
     with pytest.raises(ValueError):
         oracle.policy_grad(lp, old, adv, "ppo")
+
+
+def test_policy_grad_non_finite_inputs_and_overflowing_ratio():
+    """Rows with a non-finite old logprob or advantage carry no signal (0); a
+    ratio that overflows float64 saturates the CISPO weight at 1 + eps_high,
+    is clipped for A >= 0 and gives an infinite gradient for A < 0 in the
+    clipped surrogate (d(r A)/dlogprob = r A is unbounded there)."""
+    lp = np.array([-1.0, -1.0, -1.0, -1.0, -0.5, -0.5])
+    old = np.array([np.nan, -np.inf, -1.0, -2.0, -1000.0, -1000.0])
+    adv = np.array([1.0, 1.0, np.inf, np.nan, 1.0, -1.0])
+    c = oracle.policy_grad(lp, old, adv, "cispo", 0.2, 0.3, 1.0)
+    assert c.tolist()[:4] == [0.0, 0.0, 0.0, 0.0]
+    assert c[4] == -1.3 and c[5] == 1.3  # r = e^999.5 overflows: weight 1 + eps_high
+    k = oracle.policy_grad(lp, old, adv, "clipped", 0.2, 0.3, 1.0)
+    assert k.tolist()[:5] == [0.0, 0.0, 0.0, 0.0, 0.0]
+    assert k[5] == math.inf
+    z = oracle.policy_grad(lp, old, adv, "clipped", 0.2, 0.3, 0.0)  # scale 0: no signal
+    assert not z.any()
