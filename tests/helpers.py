@@ -50,24 +50,27 @@ def near_gap_rows(s: np.ndarray, rows: dict, eps: float = GAP_EPS) -> np.ndarray
 
 
 def compare_logprob(gpu_lp: np.ndarray, ora_lp: np.ndarray, flagged: np.ndarray):
-    """Returns (n_bad, n_flagged_mismatch, max_abs_err_on_unflagged_finite).
+    """Returns (n_bad, n_flagged_flips, max_abs_err).
 
-    A row mismatches when the GPU value is NaN, when a finite pair is further
-    apart than LOGPROB_ATOL, or when the target is inside the support on one
-    side only. Mismatches on rows whose oracle thresholds sit within GAP_EPS
-    of a decision boundary are counted and reported (the fp32 logits may
-    legitimately cross such a boundary); any other mismatch is a failure.
+    Every row whose target is inside the support on both sides has its finite
+    logprobs compared within LOGPROB_ATOL, flagged or not: a support that
+    differs by a near-tie token moves LSE_S by about that token's share of the
+    mass, far below the tolerance. Only a target membership flip (inside the
+    support on one side, outside on the other) is excused, and only on rows
+    whose oracle thresholds sit within GAP_EPS of a decision boundary; those
+    are counted in n_flagged_flips. A NaN is always a failure. max_abs_err is
+    over every row compared.
     """
     gpu_lp = np.asarray(gpu_lp, np.float64)
+    ora_lp = np.asarray(ora_lp, np.float64)
     gi = np.isneginf(gpu_lp)
     oi = np.isneginf(ora_lp)
-    both = ~gi & ~oi
+    both = ~gi & ~oi & ~np.isnan(gpu_lp)
     err = np.where(both, np.abs(gpu_lp - ora_lp), 0.0)
-    mism = (both & (err > LOGPROB_ATOL)) | np.isnan(gpu_lp) | (gi != oi)
-    n_bad = int((mism & ~flagged).sum())
-    sel = both & ~flagged
-    max_err = float(err[sel].max()) if sel.any() else 0.0
-    return n_bad, int((mism & flagged).sum()), max_err
+    flip = gi != oi
+    bad = (both & (err > LOGPROB_ATOL)) | np.isnan(gpu_lp) | (flip & ~flagged)
+    max_err = float(err[both].max()) if both.any() else 0.0
+    return int(bad.sum()), int((flip & flagged).sum()), max_err
 
 
 def grad_rows(gpu_flags: np.ndarray, ref_in_support: np.ndarray) -> np.ndarray:
@@ -91,3 +94,72 @@ def small_case(seed, T, d, V, tau=(0.5, 1.5), k_choices=(0, 50), p_choices=(1.0,
     }
     u = rng.random(T)
     return H, W, rows, u
+
+
+# --------------------------------------------------------------------------
+# the oracle's per-row loops over a process pool (spawn: the parent may
+# already hold a CUDA context, and a forked child of it would hang)
+
+
+def _oracle_call(name, args, kwargs):
+    return getattr(oracle, name)(*args, **kwargs)
+
+
+class OraclePool:
+    """Runs an oracle function on row slices in parallel and joins the
+    results in row order. The oracle itself is unchanged: each worker calls
+    the same function on a contiguous block of rows."""
+
+    def __init__(self, workers=None):
+        import concurrent.futures
+        import multiprocessing
+        import os
+
+        n = workers or max(1, min(16, (os.cpu_count() or 2) - 1))
+        self.n = n
+        self.ex = concurrent.futures.ProcessPoolExecutor(
+            max_workers=n, mp_context=multiprocessing.get_context("spawn"))
+
+    def close(self):
+        self.ex.shutdown(wait=True, cancel_futures=True)
+
+    def _slices(self, T):
+        step = max(1, -(-T // (2 * self.n)))
+        return [(a, min(T, a + step)) for a in range(0, T, step)]
+
+    @staticmethod
+    def _rows_slice(rows, a, b):
+        return {k: np.asarray(v)[a:b] for k, v in rows.items()}
+
+    def map_rows(self, name, s, rows, *extra, per_row_extra=()):
+        """oracle.<name>(s[a:b], rows[a:b], *extra[a:b] ...) for row blocks;
+        returns the per-block results in order."""
+        T = s.shape[0]
+        futs = []
+        for a, b in self._slices(T):
+            args = [s[a:b], self._rows_slice(rows, a, b)]
+            args += [np.asarray(e)[a:b] for e in per_row_extra]
+            args += list(extra)
+            futs.append(self.ex.submit(_oracle_call, name, tuple(args), {}))
+        return [f.result() for f in futs]
+
+    def forward(self, s, rows):
+        futs = []
+        for a, b in self._slices(s.shape[0]):
+            futs.append(self.ex.submit(_oracle_call, "forward",
+                                       (None, None, self._rows_slice(rows, a, b)), {"s": s[a:b]}))
+        parts = [f.result() for f in futs]
+        return {k: np.concatenate([p[k] for p in parts]) for k in parts[0]}
+
+    def filter_rows(self, s, rows):
+        parts = self.map_rows("filter_rows", s, rows)
+        return {k: np.concatenate([p[k] for p in parts]) for k in parts[0]}
+
+    def row_gaps(self, s, rows):
+        return np.concatenate(self.map_rows("row_gaps", s, rows))
+
+    def sample_rows(self, s, rows, u):
+        return np.concatenate(self.map_rows("sample_rows", s, rows, per_row_extra=(u,)))
+
+    def logit_grad(self, s, rows, g):
+        return np.concatenate(self.map_rows("logit_grad", s, rows, per_row_extra=(g,)))

@@ -1,9 +1,22 @@
 """Parity at the full sizes of the three large workloads, in the launch
-configuration the benchmark times (default row and vocabulary chunks, all
-rows on the GPU), checked on a seeded sample of rows the oracle computes one
-by one: logprobs, support sizes, dH rows and dW on a sample of vocabulary rows
-(the upstream gradient is zero outside the sampled rows so dW stays
-comparable)."""
+configuration the benchmark times (default row chunk, the workload's vocabulary
+chunk, all rows on the GPU), on a seeded sample of N_TILES whole 128-row tiles
+(512 rows) that the float64 oracle computes row by row.
+
+Checks, each able to fail on any sampled row:
+  1. logprob: within 2e-3 of the oracle on every row whose target is in the
+     support on both sides; a target-membership flip only on a row whose
+     oracle threshold lies within 1e-4 of its decision boundary (counted);
+  2. support size equal to the oracle's on every row that is not near-gap;
+  3. the forward's cuts (support size, cut id, cut logit) bit-exact against
+     the oracle's support program run on the GPU's own fp32 logits of the
+     same rows (same fp32 values, every decision in float64 on both sides);
+     a difference is only allowed where that row's top-p crossing is within
+     1e-12 of a boundary (float64 summation order);
+  4. dH on the sampled rows and dW on ~1000 sampled vocabulary rows (the
+     upstream gradient is 1 on the sampled rows whose membership agrees, 0
+     elsewhere, so dW stays comparable): relative Frobenius error < 1e-2.
+"""
 
 import numpy as np
 import pytest
@@ -11,67 +24,79 @@ import torch
 
 import oracle
 import workloads
-from helpers import (GRAD_RTOL, bf16_tensor, compare_logprob, f32_values, grad_rows,
-                     near_gap_rows, rel_fro)
+from helpers import (GAP_EPS, GRAD_RTOL, OraclePool, bf16_tensor, compare_logprob, f32_values,
+                     grad_rows, rel_fro)
 
 pytestmark = pytest.mark.gpu
 
-N_ROWS = 48
+N_TILES = 4  # 128-row tiles: 512 sampled rows
 N_VOCAB = 1024
 
 
-def _sample_rows(data, T, rng):
-    idx = set(rng.choice(T, N_ROWS, replace=False).tolist())
-    # make sure each metadata class appears
-    for key in ("top_k", "top_p", "min_p"):
-        vals = data[key]
-        for v in np.unique(vals)[:4]:
-            hits = np.flatnonzero(vals == v)
-            idx.add(int(hits[rng.integers(0, len(hits))]))
-    return np.array(sorted(idx), dtype=np.int64)
+@pytest.fixture(scope="module")
+def pool():
+    p = OraclePool()
+    yield p
+    p.close()
 
 
 @pytest.mark.parametrize("index", [3, 4, 5])
-def test_full_size_workload(cuda_lib, index):
+def test_full_size_workload(cuda_lib, pool, index):
     sts = cuda_lib
     data = workloads.make(index)
     wl = data["workload"]
     T, d, V = wl.T, wl.d, wl.V
     rng = np.random.Generator(np.random.PCG64(3000 + index))
-    sel = _sample_rows(data, T, rng)
+    tiles = np.sort(rng.choice(T // 128, N_TILES, replace=False))
+    sel = (tiles[:, None] * 128 + np.arange(128)[None, :]).reshape(-1)
     meta_sel = {k: data[k][sel] for k in ("temperature", "top_k", "top_p", "min_p")}
 
+    # the oracle: float64 logits of the sampled rows, replayed tokens drawn
+    # from its own filtered distribution, forward and threshold gaps
     Hf_sel = f32_values(data["H"][sel])
     Wf = f32_values(data["W"])
     s_sel = oracle.scaled_logits(Hf_sel, Wf, meta_sel["temperature"], vocab_slice=16384)
-    y_sel = oracle.sample_rows(s_sel, dict(meta_sel, target=np.zeros(len(sel), np.int64)),
-                               data["u"][sel])
+    rows0 = dict(meta_sel, target=np.zeros(len(sel), np.int64))
+    y_sel = pool.sample_rows(s_sel, rows0, data["u"][sel])
     rows_sel = dict(meta_sel, target=y_sel)
-    ref = oracle.forward(None, None, rows_sel, s=s_sel)
+    ref = pool.forward(s_sel, rows_sel)
+    flagged = pool.row_gaps(s_sel, rows_sel).min(axis=1) < GAP_EPS
 
+    # the GPU forward on every row (targets outside the sample are token 0)
     target = np.zeros(T, np.int64)
     target[sel] = y_sel
-
     Hd, Wd = bf16_tensor(data["H"]), bf16_tensor(data["W"])
     dev = lambda a, dt: torch.from_numpy(np.asarray(a, dt)).cuda()  # noqa: E731
     y_t = dev(target, np.int64)
     tau, k, p, mu = (dev(data["temperature"], np.float32), dev(data["top_k"], np.int32),
                      dev(data["top_p"], np.float32), dev(data["min_p"], np.float32))
     lp, saved, _ = sts.sts_forward(Hd, Wd, y_t, tau, k, p, mu, check=True)
-
     lp_sel = lp.cpu().numpy()[sel]
-    flagged = near_gap_rows(s_sel, rows_sel)
-    bad, flagged_mism, max_err = compare_logprob(lp_sel, ref["logprob"], flagged)
-    size = saved["support_size"].cpu().numpy()[sel]
-    dsize = np.abs(size - ref["size"])
-    print(f"workload {index}: {len(sel)} rows, {int(flagged.sum())} near-gap, "
-          f"{flagged_mism} near-gap membership flips, max |dlogprob| {max_err:.2e}, "
-          f"max support-size difference {int(dsize.max())} tokens")
-    assert bad == 0
-    assert not ((dsize != 0) & ~flagged).any()
+    sv = {n: v.cpu().numpy()[sel] for n, v in saved.items()}
 
-    # gradients on the rows whose target membership agrees; zero elsewhere
-    same = grad_rows(saved["flags"].cpu().numpy()[sel], ref["in_support"])
+    # 1 and 2: against the float64 oracle
+    bad, flips, max_err = compare_logprob(lp_sel, ref["logprob"], flagged)
+    dsize = np.abs(sv["support_size"] - ref["size"])
+    # 3: the forward's cuts against the oracle's program on the GPU's logits
+    S_gpu = torch.cat([sts.sts_scaled_logits(Hd, Wd, tau, t0=int(t) * 128, rows=128)
+                       for t in tiles]).cpu().numpy()
+    own = pool.filter_rows(S_gpu, rows_sel)
+    own_gap_p = pool.row_gaps(S_gpu, rows_sel)[:, 1]
+    cut_diff = ((sv["support_size"] != own["size"]) | (sv["cut_id"] != own["cut_id"])
+                | (sv["cut_logit"] != own["cut_value"].astype(np.float32)))
+    n = len(sel)
+    print(f"workload {index}: {n} rows; logprob compared on {n - flips} rows (max |dlogprob| "
+          f"{max_err:.2e}); {int((~flagged).sum())} rows with every threshold further than "
+          f"{GAP_EPS:g} from its boundary, {int(flagged.sum())} near-gap ({flips} target-membership "
+          f"flips, max support-size difference {int(dsize[flagged].max(initial=0))} tokens); "
+          f"cuts bit-exact against the oracle on the GPU's fp32 logits on "
+          f"{int((~cut_diff).sum())} of {n} rows")
+    assert bad == 0
+    assert not ((dsize != 0) & ~flagged).any(), np.flatnonzero((dsize != 0) & ~flagged)
+    assert not (cut_diff & ~(own_gap_p < 1e-12)).any(), np.flatnonzero(cut_diff)
+
+    # 4: gradients on the rows whose target membership agrees; zero elsewhere
+    same = grad_rows(sv["flags"], ref["in_support"])
     g = np.zeros(T, np.float32)
     g[sel[same]] = 1.0
     dH, dW = sts.sts_backward(Hd, Wd, y_t, tau, k, p, mu, saved, dev(g, np.float32),
@@ -79,9 +104,9 @@ def test_full_size_workload(cuda_lib, index):
     vocab = np.unique(np.concatenate([rng.choice(V, N_VOCAB, replace=False), y_sel]))
     if index == 5:
         vocab = np.unique(np.concatenate([vocab, data["dup_dst"][:64], data["dup_src"][:64]]))
-    dH_ref, dW_ref = oracle.backward(Hf_sel, Wf, rows_sel, same.astype(np.float64), s=s_sel,
-                                     vocab_rows=vocab, vocab_slice=16384)
-    dH_sel = dH.cpu().numpy()[sel]
-    assert rel_fro(dH_sel, dH_ref) < GRAD_RTOL
+    dZ = pool.logit_grad(s_sel, rows_sel, same.astype(np.float64))
+    dH_ref, dW_ref = oracle.backward(Hf_sel, Wf, rows_sel, None, vocab_rows=vocab,
+                                     vocab_slice=16384, dZ=dZ)
+    assert rel_fro(dH.cpu().numpy()[sel], dH_ref) < GRAD_RTOL
     dW_sub = dW[torch.from_numpy(vocab).cuda()].cpu().numpy()
     assert rel_fro(dW_sub, dW_ref) < GRAD_RTOL
