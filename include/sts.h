@@ -172,7 +172,8 @@ sts_status sts_filter_logits(const sts_shape* shape, const float* scaled_logits,
  * All calls share the array, which keeps the last call's contents (the header
  * is cleared at the start of each call): calls that overlap on the GPU -- on
  * different streams, or from different host threads -- race. Row-value
- * errors show per row (support_size 0, cut_id -1, cut_logit NaN); there is
+ * errors, and a row whose exact search exceeds an internal bound, show per
+ * row (support_size 0, cut_id -1, cut_logit NaN, mask row all 0); there is
  * no status word to read back. Allocates nothing. */
 sts_status sts_filter_logits_noalloc(const sts_shape* shape, const float* scaled_logits,
                                      const sts_rows* rows, int32_t* support_size,

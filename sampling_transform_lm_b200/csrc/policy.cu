@@ -12,7 +12,11 @@
 //
 // with r_t = exp(logprob_t - old_logprob_t) evaluated in float64. A row whose
 // logprob is not finite (-inf: the replayed token is outside the support;
-// NaN: an invalid row) gets 0.
+// NaN: an invalid row), or whose old logprob or advantage is not finite,
+// gets 0, and so does a row with scale * A_t == 0. r_t may overflow to +inf
+// (logprob_t - old_logprob_t > ~709.8): CISPO's weight is then 1 + eps_high,
+// the clipped surrogate is clipped for A_t >= 0 and gives an infinite
+// gradient for A_t < 0 (the objective is unbounded there).
 #include <cmath>
 
 #include "sts_internal.h"
@@ -27,11 +31,11 @@ __global__ void policy_grad_kernel(int64_t T, const float* __restrict__ logprob,
                                    float* __restrict__ grad) {
   for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T;
        t += (int64_t)gridDim.x * blockDim.x) {
-    const float lp = logprob[t];
+    const float lp = logprob[t], old = old_logprob[t], adv = advantage[t];
     double g = 0.0;
-    if (isfinite(lp)) {
-      const double a = (double)advantage[t];
-      const double r = exp((double)lp - (double)old_logprob[t]);
+    if (isfinite(lp) && isfinite(old) && isfinite(adv) && scale * (double)adv != 0.0) {
+      const double a = (double)adv;
+      const double r = exp((double)lp - (double)old);
       if (objective == STS_PG_CISPO) {
         g = -scale * a * fmin(r, 1.0 + eps_high);
       } else {

@@ -1482,15 +1482,21 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
     bool ok = resolve_row_fast<VEC>(sm, x, V, m, k, p, mu, kt, best);
     if (!ok) ok = resolve_row_exact<VEC>(sm, x, V, m, k, p, mu, kt, hist_valid, best);
 
-    if (!ok) {
+    if (!ok) {  // a bound of the exact search was exceeded: the row fails like an invalid one
       if (threadIdx.x == 0) {
         atomicCAS(&a.hdr->err, 0, (int)STS_ERR_OVERFLOW);
         const float nan = __int_as_float(0x7fc00000);
         if (a.logprob) a.logprob[r] = nan;
+        if (a.row_max) a.row_max[r] = nan;
+        if (a.lse_support) a.lse_support[r] = nan;
+        if (a.cut_logit) a.cut_logit[r] = nan;
+        if (a.cut_id) a.cut_id[r] = -1;
         if (a.sampled) a.sampled[r] = -1;
         if (a.support_size) a.support_size[r] = 0;
         if (a.flags_out) a.flags_out[r] = STS_ROW_INVALID;
       }
+      if (a.mask)
+        for (int i = threadIdx.x; i < V; i += RT) a.mask[(size_t)r * V + i] = 0;
       __syncthreads();
       continue;
     }
