@@ -7,6 +7,7 @@ from .sts_oracle import (  # noqa: F401
     filter_rows,
     forward,
     logit_grad,
+    logprob_on_prefix,
     policy_grad,
     row_gaps,
     sample_rows,

@@ -71,6 +71,9 @@ __all__ = [
     "backward",
     "sample_rows",
     "row_gaps",
+    "logprob_on_prefix",
+    "logit_grad",
+    "policy_grad",
 ]
 
 
@@ -238,6 +241,33 @@ def forward(H, W, rows, s=None):
         res["in_support"][t] = inside
         res["logprob"][t] = min(float(s[t, y[t]]) - lse, 0.0) if inside else -math.inf
     return res
+
+
+def logprob_on_prefix(s, rows, sizes):
+    """Selected-token logprob when row t's support is the first sizes[t]
+    positions of its (s desc, id asc) order; returns (logprob, in_support).
+
+    The same definition as ``forward`` ([xorl#74] item 2, item 4, the <= 0
+    clamp of "Self-review pass") with the support size given instead of
+    derived. A result whose support differs from the oracle's at a near-tie
+    boundary is a valid alternative; its logprob is then fixed by that
+    support, and this gives it.
+    """
+    s = np.asarray(s, dtype=np.float64)
+    T, V = s.shape
+    y = np.asarray(rows["target"], dtype=np.int64)
+    lp = np.zeros(T, dtype=np.float64)
+    inside = np.zeros(T, dtype=bool)
+    for t in range(T):
+        size = int(sizes[t])
+        order = np.argsort(-s[t], kind="stable")
+        ss = s[t, order]
+        lse = _support_lse(ss, float(ss[0]), size)
+        rank = np.empty(V, dtype=np.int64)
+        rank[order] = np.arange(V)
+        inside[t] = bool(rank[y[t]] < size)
+        lp[t] = min(float(s[t, y[t]]) - lse, 0.0) if inside[t] else -math.inf
+    return lp, inside
 
 
 def logit_grad(s, rows, grad_logprob):

@@ -49,28 +49,33 @@ def near_gap_rows(s: np.ndarray, rows: dict, eps: float = GAP_EPS) -> np.ndarray
     return oracle.row_gaps(s, rows).min(axis=1) < eps
 
 
-def compare_logprob(gpu_lp: np.ndarray, ora_lp: np.ndarray, flagged: np.ndarray):
-    """Returns (n_bad, n_flagged_flips, max_abs_err).
+def compare_logprob(gpu_lp, gpu_size, s, rows, ref, flagged):
+    """Returns (n_bad, n_size_diff, max_abs_err). Every row is compared.
 
-    Every row whose target is inside the support on both sides has its finite
-    logprobs compared within LOGPROB_ATOL, flagged or not: a support that
-    differs by a near-tie token moves LSE_S by about that token's share of the
-    mass, far below the tolerance. Only a target membership flip (inside the
-    support on one side, outside on the other) is excused, and only on rows
-    whose oracle thresholds sit within GAP_EPS of a decision boundary; those
-    are counted in n_flagged_flips. A NaN is always a failure. max_abs_err is
-    over every row compared.
+    The expected logprob of a row is the oracle's, or -- where the GPU's
+    support size differs from the oracle's, which is only allowed on a row
+    whose oracle threshold lies within GAP_EPS of a decision boundary -- the
+    oracle's logprob on the GPU's support (``oracle.logprob_on_prefix``): the
+    order of the row is unique, so a support is a prefix length, and the
+    logprob follows from it. On every row the target membership must agree
+    with that expectation and finite values must agree within LOGPROB_ATOL;
+    a NaN is always a failure.
     """
     gpu_lp = np.asarray(gpu_lp, np.float64)
-    ora_lp = np.asarray(ora_lp, np.float64)
+    gpu_size = np.asarray(gpu_size, np.int64)
+    want = np.array(ref["logprob"], np.float64)
+    diff = gpu_size != np.asarray(ref["size"])
+    if diff.any():
+        idx = np.flatnonzero(diff)
+        sub = {k: np.asarray(v)[idx] for k, v in rows.items()}
+        want[idx] = oracle.logprob_on_prefix(np.asarray(s)[idx], sub, gpu_size[idx])[0]
     gi = np.isneginf(gpu_lp)
-    oi = np.isneginf(ora_lp)
-    both = ~gi & ~oi & ~np.isnan(gpu_lp)
-    err = np.where(both, np.abs(gpu_lp - ora_lp), 0.0)
-    flip = gi != oi
-    bad = (both & (err > LOGPROB_ATOL)) | np.isnan(gpu_lp) | (flip & ~flagged)
+    wi = np.isneginf(want)
+    both = ~gi & ~wi & ~np.isnan(gpu_lp)
+    err = np.where(both, np.abs(gpu_lp - want), 0.0)
+    bad = (both & (err > LOGPROB_ATOL)) | np.isnan(gpu_lp) | (gi != wi) | (diff & ~flagged)
     max_err = float(err[both].max()) if both.any() else 0.0
-    return int(bad.sum()), int((flip & flagged).sum()), max_err
+    return int(bad.sum()), int(diff.sum()), max_err
 
 
 def grad_rows(gpu_flags: np.ndarray, ref_in_support: np.ndarray) -> np.ndarray:

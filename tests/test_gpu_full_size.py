@@ -4,18 +4,21 @@ chunk, all rows on the GPU), on a seeded sample of N_TILES whole 128-row tiles
 (512 rows) that the float64 oracle computes row by row.
 
 Checks, each able to fail on any sampled row:
-  1. logprob: within 2e-3 of the oracle on every row whose target is in the
-     support on both sides; a target-membership flip only on a row whose
-     oracle threshold lies within 1e-4 of its decision boundary (counted);
-  2. support size equal to the oracle's on every row that is not near-gap;
+  1. support size equal to the oracle's on every row that is not near-gap
+     (every threshold that can move the support further than 1e-4 from its
+     boundary); a near-gap row may take another valid size (counted);
+  2. logprob and target membership on every row: against the oracle's, or,
+     where the support size legitimately differs, against the oracle's
+     logprob on the GPU's support (within 2e-3);
   3. the forward's cuts (support size, cut id, cut logit) bit-exact against
      the oracle's support program run on the GPU's own fp32 logits of the
      same rows (same fp32 values, every decision in float64 on both sides);
      a difference is only allowed where that row's top-p crossing is within
      1e-12 of a boundary (float64 summation order);
   4. dH on the sampled rows and dW on ~1000 sampled vocabulary rows (the
-     upstream gradient is 1 on the sampled rows whose membership agrees, 0
-     elsewhere, so dW stays comparable): relative Frobenius error < 1e-2.
+     upstream gradient is 1 on the sampled rows whose support equals the
+     oracle's, 0 elsewhere, so dW stays comparable): relative Frobenius
+     error < 1e-2.
 """
 
 import numpy as np
@@ -75,7 +78,7 @@ def test_full_size_workload(cuda_lib, pool, index):
     sv = {n: v.cpu().numpy()[sel] for n, v in saved.items()}
 
     # 1 and 2: against the float64 oracle
-    bad, flips, max_err = compare_logprob(lp_sel, ref["logprob"], flagged)
+    bad, ndiff, max_err = compare_logprob(lp_sel, sv["support_size"], s_sel, rows_sel, ref, flagged)
     dsize = np.abs(sv["support_size"] - ref["size"])
     # 3: the forward's cuts against the oracle's program on the GPU's logits
     S_gpu = torch.cat([sts.sts_scaled_logits(Hd, Wd, tau, t0=int(t) * 128, rows=128)
@@ -85,18 +88,17 @@ def test_full_size_workload(cuda_lib, pool, index):
     cut_diff = ((sv["support_size"] != own["size"]) | (sv["cut_id"] != own["cut_id"])
                 | (sv["cut_logit"] != own["cut_value"].astype(np.float32)))
     n = len(sel)
-    print(f"workload {index}: {n} rows; logprob compared on {n - flips} rows (max |dlogprob| "
+    print(f"workload {index}: {n} rows; logprob compared on all {n} (max |dlogprob| "
           f"{max_err:.2e}); {int((~flagged).sum())} rows with every threshold further than "
-          f"{GAP_EPS:g} from its boundary, {int(flagged.sum())} near-gap ({flips} target-membership "
-          f"flips, max support-size difference {int(dsize[flagged].max(initial=0))} tokens); "
+          f"{GAP_EPS:g} from its boundary, {int(flagged.sum())} near-gap ({ndiff} with another "
+          f"valid support size, at most {int(dsize.max(initial=0))} tokens apart); "
           f"cuts bit-exact against the oracle on the GPU's fp32 logits on "
           f"{int((~cut_diff).sum())} of {n} rows")
     assert bad == 0
-    assert not ((dsize != 0) & ~flagged).any(), np.flatnonzero((dsize != 0) & ~flagged)
     assert not (cut_diff & ~(own_gap_p < 1e-12)).any(), np.flatnonzero(cut_diff)
 
-    # 4: gradients on the rows whose target membership agrees; zero elsewhere
-    same = grad_rows(sv["flags"], ref["in_support"])
+    # 4: gradients on the rows whose support equals the oracle's; zero elsewhere
+    same = grad_rows(sv["flags"], ref["in_support"]) & (dsize == 0)
     g = np.zeros(T, np.float32)
     g[sel[same]] = 1.0
     dH, dW = sts.sts_backward(Hd, Wd, y_t, tau, k, p, mu, saved, dev(g, np.float32),
