@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define STS_ABI_VERSION 1
+#define STS_ABI_VERSION 2
 
 /* cudaStream_t without pulling in the CUDA headers (same opaque type). */
 typedef struct CUstream_st* sts_stream_t;
@@ -123,11 +123,16 @@ size_t sts_workspace_bytes(const sts_shape* shape, int pass);
  * chunk size. */
 int64_t sts_vocab_chunk(const sts_shape* shape);
 
-/* Forward: logprob[T] (fp32) and the saved per-row scalars.
- * ws must hold sts_workspace_bytes(shape, 0) bytes. */
+/* Forward: logprob[T] (fp32) and the saved per-row scalars; optionally the
+ * entropy of each row's filtered distribution, entropy[T] (fp32, nats:
+ * H_t = -sum_{i in S_t} p_i ln p_i, p_i = exp(s_i - LSE_S); "align
+ * architecture v2: proposal", section 5.4 A, entropy from the same sweep),
+ * formed from the same per-logit float64 masses as LSE_S (one more float64
+ * sum per logit); entropy may be NULL (then nothing extra is computed).
+ * Invalid rows get NaN. ws must hold sts_workspace_bytes(shape, 0) bytes. */
 sts_status sts_forward(const sts_shape* shape, const void* H_bf16, const void* W_bf16,
-                       const sts_rows* rows, float* logprob, const sts_saved* saved,
-                       void* ws, size_t ws_bytes, sts_stream_t stream);
+                       const sts_rows* rows, float* logprob, float* entropy,
+                       const sts_saved* saved, void* ws, size_t ws_bytes, sts_stream_t stream);
 
 /* Backward: dH[T,d] and dW[V,d] (fp32) from grad_logprob[T] and the scalars
  * saved by sts_forward on the same H, W and rows. dH is overwritten; dW is
@@ -137,6 +142,33 @@ sts_status sts_backward(const sts_shape* shape, const void* H_bf16, const void* 
                         const sts_rows* rows, const sts_saved* saved,
                         const float* grad_logprob, float* dH, float* dW, int accumulate_dW,
                         void* ws, size_t ws_bytes, sts_stream_t stream);
+
+/* Receives one finished slice of the weight gradient: rows [v0, v0 + rows) of
+ * dW, which start at dW_slice (device memory, row-major [rows, d] fp32). */
+typedef void (*sts_slice_fn)(void* user, int64_t v0, int64_t rows, float* dW_slice,
+                             sts_stream_t stream);
+
+/* sts_backward for data-parallel training: the weight gradient is written once
+ * per vocabulary slice ("Self-review pass" of the xorl PR) and its partial sums
+ * must be added across the ranks that scored other rows ("What this PR does",
+ * item 2). Right after the GEMM that writes slice [v0, v0 + rows) has been
+ * enqueued on `stream`, and before anything else is enqueued, on_dw_slice is
+ * called on the calling host thread, once per slice in increasing v0. The
+ * callee typically records an event on `stream`, makes a communication stream
+ * wait for it and enqueues the slice's all-reduce (or reduce-scatter) there,
+ * so that the exchange of slice i overlaps the dH GEMM of slice i and the
+ * GEMMs of slice i + 1; it must make `stream` wait for its exchanges before
+ * dW is read. The library writes no element of a slice after handing it out.
+ * The GEMMs are persistent (one CTA per SM) and would hold every SM for
+ * their whole run, so comm_sms SMs (0 <= comm_sms < SM count, else
+ * STS_ERR_SHAPE) are left free for the exchange kernels. on_dw_slice == NULL
+ * with comm_sms == 0 is sts_backward. The callback must not call back into
+ * the library on the same workspace. */
+sts_status sts_backward_sliced(const sts_shape* shape, const void* H_bf16, const void* W_bf16,
+                               const sts_rows* rows, const sts_saved* saved,
+                               const float* grad_logprob, float* dH, float* dW, int accumulate_dW,
+                               void* ws, size_t ws_bytes, sts_stream_t stream,
+                               sts_slice_fn on_dw_slice, void* user, int comm_sms);
 
 /* Draw one token per row from the filtered distribution: the inverse CDF of
  * the support walked in (s desc, id asc) order, taking the first kept token
@@ -150,12 +182,13 @@ sts_status sts_sample(const sts_shape* shape, const void* H_bf16, const void* W_
 
 /* Test hook: run only the support program on caller-given fp32 scaled logits
  * [T, V] (row stride V). Writes support_size, cut_logit, cut_id per row and,
- * when mask is not NULL, mask[T, V] (1 = kept). rows->target is ignored.
- * ws: sts_workspace_bytes(shape, 2). */
+ * when mask is not NULL, mask[T, V] (1 = kept); when entropy is not NULL, the
+ * entropy of each row's filtered distribution as sts_forward forms it.
+ * rows->target is ignored. ws: sts_workspace_bytes(shape, 2). */
 sts_status sts_filter_logits(const sts_shape* shape, const float* scaled_logits,
                              const sts_rows* rows, int32_t* support_size, float* cut_logit,
-                             int32_t* cut_id, uint8_t* mask, void* ws, size_t ws_bytes,
-                             sts_stream_t stream);
+                             int32_t* cut_id, uint8_t* mask, float* entropy, void* ws,
+                             size_t ws_bytes, sts_stream_t stream);
 
 /* sts_filter_logits for callers that cannot allocate device memory: code
  * running under a fixed device-memory reservation (where cudaMalloc may fail,
@@ -199,6 +232,15 @@ sts_status sts_probe_mass_exp(const float* s, float m, double* mass, double* lib
 /* Synchronise the stream and read the status word a previous call left in
  * ws. first_bad_row (may be NULL) receives the lowest failing row or -1. */
 sts_status sts_get_status(const void* ws, sts_stream_t stream, int64_t* first_bad_row);
+
+/* Diagnostic: how many rows the support resolver decided by each of its
+ * paths since the workspace's last reset (every sts_forward, sts_sample and
+ * sts_filter_logits call resets it): counts[0] the planned pass (a sampled
+ * plan confirmed by one exact pass), counts[1] the fast path (full count
+ * histogram, then an exact pass), counts[2] the exact search, counts[3]
+ * identity rows (one pass). Synchronises the stream. counts: 4 int64 on the
+ * host. Not from the pages: a measure of where the resolver's time goes. */
+sts_status sts_path_counts(const void* ws, sts_stream_t stream, int64_t* counts);
 
 /* Policy-gradient objectives for sts_policy_grad. */
 typedef enum { STS_PG_CISPO = 0, STS_PG_CLIPPED = 1 } sts_pg_objective;

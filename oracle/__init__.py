@@ -3,6 +3,7 @@
 from .sts_oracle import (  # noqa: F401
     RowFilter,
     backward,
+    entropy,
     filter_row,
     filter_rows,
     forward,

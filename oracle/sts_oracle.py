@@ -72,6 +72,7 @@ __all__ = [
     "sample_rows",
     "row_gaps",
     "logprob_on_prefix",
+    "entropy",
     "logit_grad",
     "policy_grad",
 ]
@@ -241,6 +242,32 @@ def forward(H, W, rows, s=None):
         res["in_support"][t] = inside
         res["logprob"][t] = min(float(s[t, y[t]]) - lse, 0.0) if inside else -math.inf
     return res
+
+
+def entropy(s, rows, sizes=None):
+    """Entropy of each row's filtered (renormalised) distribution, in nats:
+    H_t = -sum_{i in S_t} p_i ln p_i with p_i = exp(s_i - LSE_S). ``sizes``
+    (optional) gives each row's support size instead of deriving it, as
+    ``logprob_on_prefix`` does.
+
+    [align-v2] section 5.4 A names the per-token entropy as one of the
+    statistics of the fused head ("entropy from the same sweep"); the
+    distribution is the one the selected logprob is scored on ([xorl#74]
+    item 2): the support of item 1, renormalised. Written as the sum of the
+    non-negative terms p_i (LSE_S - s_i), exactly rounded (math.fsum).
+    """
+    s = np.asarray(s, dtype=np.float64)
+    T = s.shape[0]
+    out = np.zeros(T, dtype=np.float64)
+    for t in range(T):
+        k, p, mu = _row_meta(rows, t)
+        f = filter_row(s[t], k, p, mu)
+        size = f.size if sizes is None else int(sizes[t])
+        ss = s[t, f.order[:size]]
+        lse = _support_lse(ss, f.m, size)
+        pr = np.exp(ss - lse)
+        out[t] = math.fsum(pr * (lse - ss))
+    return out
 
 
 def logprob_on_prefix(s, rows, sizes):

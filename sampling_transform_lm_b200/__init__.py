@@ -21,6 +21,8 @@ import os
 
 import torch
 
+from .dp import SliceAllReduce  # noqa: E402
+
 __all__ = [
     "StsError",
     "load",
@@ -29,11 +31,13 @@ __all__ = [
     "sts_vocab_chunk",
     "sts_forward",
     "sts_backward",
+    "SliceAllReduce",
     "sts_sample",
     "sts_filter_logits",
     "sts_scaled_logits",
     "sts_policy_grad",
     "sts_get_status",
+    "sts_path_counts",
     "sts_status_string",
     "sts_probe_mass_exp",
     "sts_launch_count",
@@ -78,6 +82,8 @@ EXPORTED_SYMBOLS = (
     "sts_timing_read",
     "sts_filter_logits_noalloc",
     "sts_policy_grad",
+    "sts_path_counts",
+    "sts_backward_sliced",
 )
 
 
@@ -97,6 +103,10 @@ class _Rows(ctypes.Structure):
     _fields_ = [("len", ctypes.c_int64), ("target", ctypes.c_void_p),
                 ("temperature", ctypes.c_void_p), ("top_k", ctypes.c_void_p),
                 ("top_p", ctypes.c_void_p), ("min_p", ctypes.c_void_p)]
+
+
+_SLICE_FN = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                             ctypes.c_void_p)
 
 
 class _Saved(ctypes.Structure):
@@ -126,21 +136,27 @@ def load():
     lib.sts_workspace_bytes.restype = S
     lib.sts_vocab_chunk.argtypes = [ctypes.POINTER(_Shape)]
     lib.sts_vocab_chunk.restype = ctypes.c_int64
-    lib.sts_forward.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows), P,
+    lib.sts_forward.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows), P, P,
                                 ctypes.POINTER(_Saved), P, S, P]
     lib.sts_forward.restype = ctypes.c_int
     lib.sts_backward.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows),
                                  ctypes.POINTER(_Saved), P, P, P, ctypes.c_int, P, S, P]
     lib.sts_backward.restype = ctypes.c_int
+    lib.sts_backward_sliced.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows),
+                                        ctypes.POINTER(_Saved), P, P, P, ctypes.c_int, P, S, P,
+                                        _SLICE_FN, P, ctypes.c_int]
+    lib.sts_backward_sliced.restype = ctypes.c_int
     lib.sts_sample.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows), P, P, P, S, P]
     lib.sts_sample.restype = ctypes.c_int
     lib.sts_filter_logits.argtypes = [ctypes.POINTER(_Shape), P, ctypes.POINTER(_Rows), P, P, P, P,
-                                      P, S, P]
+                                      P, P, S, P]
     lib.sts_filter_logits.restype = ctypes.c_int
     lib.sts_scaled_logits.argtypes = [ctypes.POINTER(_Shape), P, P, P, I64, I64, I64, I64, P, I64, P]
     lib.sts_scaled_logits.restype = ctypes.c_int
     lib.sts_get_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
     lib.sts_get_status.restype = ctypes.c_int
+    lib.sts_path_counts.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
+    lib.sts_path_counts.restype = ctypes.c_int
     lib.sts_status_string.argtypes = [ctypes.c_int]
     lib.sts_status_string.restype = ctypes.c_char_p
     lib.sts_probe_mass_exp.argtypes = [P, ctypes.c_float, P, P, I64, P]
@@ -257,11 +273,13 @@ def _hw(H, W):
 
 
 def sts_forward(H, W, target, temperature, top_k, top_p, min_p, *, row_chunk=0, ws=None,
-                stream=None, check=False):
+                stream=None, check=False, entropy=False):
     """Filtered-support logprob per row plus the saved per-row scalars.
 
-    Returns ``(logprob [T] fp32, saved dict, workspace)``. With ``check`` the
-    call synchronises and raises on a row-value error.
+    Returns ``(logprob [T] fp32, saved dict, workspace)``. With ``entropy``
+    the dict also holds ``"entropy"`` [T] fp32, the entropy (nats) of each
+    row's filtered distribution. With ``check`` the call synchronises and
+    raises on a row-value error.
     """
     lib = load()
     T, d, V = _hw(H, W)
@@ -280,8 +298,11 @@ def sts_forward(H, W, target, temperature, top_k, top_p, min_p, *, row_chunk=0, 
     }
     sv = _Saved(*(_ptr(saved[k]) for k in ("row_max", "lse_support", "cut_logit", "cut_id",
                                             "support_size", "flags")))
+    ent = torch.empty(T, dtype=torch.float32, device=dev) if entropy else None
     st = lib.sts_forward(ctypes.byref(sh), _ptr(H), _ptr(W), ctypes.byref(rows), _ptr(logprob),
-                         ctypes.byref(sv), _ptr(ws), ws.numel(), _stream(stream))
+                         _ptr(ent), ctypes.byref(sv), _ptr(ws), ws.numel(), _stream(stream))
+    if ent is not None:
+        saved["entropy"] = ent
     _check(st, "sts_forward")
     if check:
         sts_get_status(ws, stream, raise_on_error=True)
@@ -290,8 +311,14 @@ def sts_forward(H, W, target, temperature, top_k, top_p, min_p, *, row_chunk=0, 
 
 def sts_backward(H, W, target, temperature, top_k, top_p, min_p, saved, grad_logprob, *,
                  dW=None, dH=None, accumulate_dW=False, vocab_chunk=0, ws=None, stream=None,
-                 check=False):
-    """dH [T, d] and dW [V, d] (fp32) of sum_t g_t * logprob_t."""
+                 check=False, on_dw_slice=None, comm_sms=0):
+    """dH [T, d] and dW [V, d] (fp32) of sum_t g_t * logprob_t.
+
+    ``on_dw_slice(v0, rows, dW_slice)`` (optional) is called on this thread,
+    in increasing v0, right after the GEMM that writes dW[v0:v0 + rows] has
+    been enqueued (``sts_backward_sliced``): a data-parallel caller starts the
+    slice's cross-rank sum there (see ``SliceAllReduce``). ``comm_sms`` SMs are
+    left free of the persistent GEMMs for the exchange kernels."""
     lib = load()
     T, d, V = _hw(H, W)
     rows = _rows(T, target, temperature, top_k, top_p, min_p)
@@ -311,10 +338,29 @@ def sts_backward(H, W, target, temperature, top_k, top_p, min_p, saved, grad_log
         _need(dW, torch.float32, "dW", (V, d))
     sv = _Saved(*(_ptr(saved[k]) for k in ("row_max", "lse_support", "cut_logit", "cut_id",
                                             "support_size", "flags")))
-    st = lib.sts_backward(ctypes.byref(sh), _ptr(H), _ptr(W), ctypes.byref(rows), ctypes.byref(sv),
-                          _ptr(grad_logprob), _ptr(dH), _ptr(dW), 1 if accumulate_dW else 0,
-                          _ptr(ws), ws.numel(), _stream(stream))
-    _check(st, "sts_backward")
+    if on_dw_slice is None and not comm_sms:
+        st = lib.sts_backward(ctypes.byref(sh), _ptr(H), _ptr(W), ctypes.byref(rows),
+                              ctypes.byref(sv), _ptr(grad_logprob), _ptr(dH), _ptr(dW),
+                              1 if accumulate_dW else 0, _ptr(ws), ws.numel(), _stream(stream))
+        _check(st, "sts_backward")
+    else:
+        errors = []
+
+        def hook(_user, v0, n, _ptr_slice, _st):
+            try:
+                if on_dw_slice is not None:
+                    on_dw_slice(int(v0), int(n), dW[v0:v0 + n])
+            except BaseException as e:  # noqa: BLE001  (re-raised after the call)
+                errors.append(e)
+
+        cb = _SLICE_FN(hook)
+        st = lib.sts_backward_sliced(ctypes.byref(sh), _ptr(H), _ptr(W), ctypes.byref(rows),
+                                     ctypes.byref(sv), _ptr(grad_logprob), _ptr(dH), _ptr(dW),
+                                     1 if accumulate_dW else 0, _ptr(ws), ws.numel(),
+                                     _stream(stream), cb, None, int(comm_sms))
+        if errors:
+            raise errors[0]
+        _check(st, "sts_backward_sliced")
     if check:
         sts_get_status(ws, stream, raise_on_error=True)
     return dH, dW
@@ -338,8 +384,10 @@ def sts_sample(H, W, temperature, top_k, top_p, min_p, u, *, row_chunk=0, ws=Non
     return out
 
 
-def sts_filter_logits(S, top_k, top_p, min_p, *, want_mask=False, ws=None, stream=None, check=False):
-    """The support program alone on fp32 scaled logits S [T, V]."""
+def sts_filter_logits(S, top_k, top_p, min_p, *, want_mask=False, want_entropy=False, ws=None,
+                      stream=None, check=False):
+    """The support program alone on fp32 scaled logits S [T, V] (with
+    ``want_entropy`` also the entropy of each row's filtered distribution)."""
     lib = load()
     _need(S, torch.float32, "S")
     T, V = S.shape
@@ -353,13 +401,14 @@ def sts_filter_logits(S, top_k, top_p, min_p, *, want_mask=False, ws=None, strea
     cut_logit = torch.empty(T, dtype=torch.float32, device=S.device)
     cut_id = torch.empty(T, dtype=torch.int32, device=S.device)
     mask = torch.empty((T, V), dtype=torch.uint8, device=S.device) if want_mask else None
+    ent = torch.empty(T, dtype=torch.float32, device=S.device) if want_entropy else None
     st = lib.sts_filter_logits(ctypes.byref(sh), _ptr(S), ctypes.byref(rows), _ptr(size),
-                               _ptr(cut_logit), _ptr(cut_id), _ptr(mask), _ptr(ws), ws.numel(),
-                               _stream(stream))
+                               _ptr(cut_logit), _ptr(cut_id), _ptr(mask), _ptr(ent), _ptr(ws),
+                               ws.numel(), _stream(stream))
     _check(st, "sts_filter_logits")
     if check:
         sts_get_status(ws, stream, raise_on_error=True)
-    return {"size": size, "cut_logit": cut_logit, "cut_id": cut_id, "mask": mask}
+    return {"size": size, "cut_logit": cut_logit, "cut_id": cut_id, "mask": mask, "entropy": ent}
 
 
 def sts_filter_logits_noalloc(S, top_k, top_p, min_p, *, support_size, cut_logit, cut_id,
@@ -471,3 +520,15 @@ def sts_get_status(ws, stream=None, raise_on_error=False):
     if raise_on_error and st != STS_OK:
         raise StsError(st, f"row {row.value}" if row.value >= 0 else "device status")
     return int(st), int(row.value)
+
+
+RESOLVE_PATHS = ("planned", "fast", "exact", "identity")
+
+
+def sts_path_counts(ws, stream=None):
+    """Rows the support resolver decided by each path since ``ws`` was last
+    reset by a forward / sample / filter call: {path: rows}. Synchronises."""
+    lib = load()
+    counts = (ctypes.c_int64 * 4)()
+    _check(lib.sts_path_counts(_ptr(ws), _stream(stream), counts), "sts_path_counts")
+    return {name: int(counts[i]) for i, name in enumerate(RESOLVE_PATHS)}

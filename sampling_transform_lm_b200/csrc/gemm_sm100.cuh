@@ -69,13 +69,18 @@ struct GemmParams {
   int* err;      // STS_ERR_TIMEOUT lands here
   float* max_part;  // kEpiLogits: per-(row, 256-column tile) max, [M][max_ld]; may be null
   int max_ld;
+  // Raster: tiles run in groups of group_m m-blocks (0: GEMM_GROUP_M), every
+  // n-block of a group before the next group, so a group's A panels are
+  // reused from L2 across its n-blocks and each B panel across its m-blocks.
+  int group_m;
 };
 
-__device__ __forceinline__ void gemm_tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
-  const int per_group = GEMM_GROUP_M * num_n;
+__device__ __forceinline__ void gemm_tile_coords(int t, int num_m, int num_n, int group_m, int& mb,
+                                                 int& nb) {
+  const int per_group = group_m * num_n;
   const int g = t / per_group;
-  const int first = g * GEMM_GROUP_M;
-  const int gm = min(GEMM_GROUP_M, num_m - first);
+  const int first = g * group_m;
+  const int gm = min(group_m, num_m - first);
   const int r = t - g * per_group;
   mb = first + r % gm;
   nb = r / gm;
@@ -107,6 +112,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int num_n = (p.N + GEMM_BN - 1) / GEMM_BN;
   const int num_tiles = num_m * num_n;
   const int nk = (p.K + GEMM_BK - 1) / GEMM_BK;
+  const int group_m = p.group_m > 0 ? p.group_m : GEMM_GROUP_M;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < GEMM_STAGES; ++s) {
@@ -143,7 +149,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     bool ok = true;
     for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
       int mb, nb;
-      gemm_tile_coords(t, num_m, num_n, mb, nb);
+      gemm_tile_coords(t, num_m, num_n, group_m, mb, nb);
       for (int kb = 0; kb < nk; ++kb) {
         if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.err)) {
           ok = false;
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int sel = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       int mb, nb;
-      gemm_tile_coords(t, num_m, num_n, mb, nb);
+      gemm_tile_coords(t, num_m, num_n, group_m, mb, nb);
       const int buf = it & 1;
       const uint32_t aphase = (uint32_t)(it >> 1) & 1u;
       if (!mbar_wait(smem_u32(&tfull[buf]), aphase, abort_flag, p.err)) break;

@@ -21,27 +21,38 @@
 //
 // Work per row (one 512-thread CTA per SM, persistent over rows; a row's
 // metadata and the projection epilogue's per-tile maxima, which give the
-// unfiltered max m, are loaded one row ahead):
+// unfiltered max m, are loaded one row ahead). Rows with a 16-byte aligned
+// start stream through a shared-memory ring filled by bulk copies (one thread
+// keeps four 16 KB chunks in flight), so no pass holds its loads in registers.
 //
-//   count pass   a 4096-bucket count histogram with buckets uniform in m - s
-//                (floor((m - s) * 128), clamped to 4095). The bucket index is
-//                monotone in s, so every bucket is a contiguous run of the
-//                order.
-//   planning     from the counts alone: the top-k cut's bucket; the top-p
-//                crossing's bucket estimated with mid-bucket weights (with a
-//                neighbour where the estimate lies within six sigma of an
-//                edge; one retry with a 3-bucket window if the exact masses
-//                then place the crossing outside); the min-p threshold's
-//                bucket and the non-empty bucket before it.
-//   exact pass   (from L2: the count pass marks the row's lines evict-last)
-//                float64 masses of every element, summed in registers (the
-//                total, the mass before the window, the mass before the min-p
-//                bucket), and the elements of the planned buckets gathered
-//                into per-warp slices of a candidate buffer, then packed.
+//   buckets      floor((m - s) * 128), clamped to 4095: monotone in s, so
+//                every bucket is a contiguous run of the order.
+//   planned path (first) a count histogram of one chunk in eight plans the
+//                range to gather: for top-k the buckets up to the k-th
+//                element, for min-p the buckets around its threshold (when
+//                top-p is on too, only where the sample puts the crossing
+//                clearly after the min-p prefix). One pass gathers that range
+//                and, for min-p, weighs and counts everything before it, and
+//                the row is decided from the gathered elements.
+//   fast path    (rows whose plan does not hold, and top-p rows) a count pass
+//                adds the rest of the row to the sample's histogram; the top-p
+//                crossing's bucket is estimated from the counts with
+//                mid-bucket weights (with a neighbour where the estimate lies
+//                within six sigma of an edge; one retry with a 3-bucket window
+//                if the exact masses then place the crossing outside), the
+//                min-p threshold's bucket and the non-empty bucket before it
+//                planned. The exact pass (from L2: the count pass marks the
+//                row's lines evict-last) forms float64 masses of every element,
+//                summed in registers (the total, the mass before the window, the
+//                mass before the min-p bucket), and gathers the planned buckets'
+//                elements into per-warp slices of a candidate buffer.
 //   finish       exact masses of the window buckets place the crossing in one
 //                bucket; its elements are sorted by composite key (a bitonic
 //                network held mostly in registers and warp shuffles) and
 //                scanned, which places each cut exactly.
+//   entropy      (when asked) each region's sum of exp(s - m) (s - m) next to
+//                its mass, in the same pass, gives the entropy of the
+//                renormalised support: ln Z_S - sum_S q (s - m) / Z_S.
 //
 // When the plan cannot be proven to hold a cut (a crossing outside the
 // window, too many candidates, large top-k) the row falls back to the exact
@@ -75,6 +86,9 @@ constexpr int SCAP = 4096;          // candidates sorted and scanned at once
 constexpr float BIN_SCALE = 128.f;  // level-0 buckets per logit unit
 constexpr int MAX_LEVELS = 8;
 constexpr int UNROLL = 4;           // float4 loads in flight per thread
+constexpr int SAMPLE_EVERY = 8;     // the planning sample reads one chunk in 8
+constexpr int CH_F4 = 2 * RT;       // float4s of a streamed chunk (two per thread)
+constexpr int NSTAGE = 4;           // chunks in flight in the shared-memory ring
 
 // exp(-b / 128) for every bucket b.
 struct ExpTab {
@@ -90,6 +104,14 @@ __device__ void init_exp_tab(ExpTab& t, int tid, int nthreads) {
 // The bucket masses (planning and the exact histogram) and the candidates'
 // mass scan are never live at once and share storage.
 struct RSmem {
+  // Rows with a 16-byte aligned start are streamed through this ring by bulk
+  // copies (one thread issues them, chunks in flight = NSTAGE).
+  float4 ring[NSTAGE][CH_F4];
+  unsigned long long full_bar[NSTAGE];   // bulk copy landed (tx bytes)
+  unsigned long long empty_bar[NSTAGE];  // every warp done with the chunk
+  int abort_flag;                        // a bounded wait gave up
+  uint32_t ring_q[RT];                   // per thread: chunks consumed so far (all equal)
+  int* err;                              // the workspace status word's error field
   union {
     double mass[NB];
     double cq[SCAP];  // inclusive mass scan of at most SCAP sorted candidates
@@ -249,6 +271,83 @@ __device__ __forceinline__ void for_each(const float* __restrict__ x, int V, F&&
     }
   }
 }
+
+// ---------------------------------------------------------------- streaming through the ring
+// A row whose start is 16-byte aligned is read in chunks of CH_F4 float4s
+// (chunk c = float4s [c CH_F4, min(V4, (c + 1) CH_F4))) that bulk copies put
+// into the shared-memory ring. Thread 0 keeps up to NSTAGE copies in flight, so
+// a pass's HBM latency is covered without holding loads in registers; every
+// thread takes the float4s at offsets t and t + RT of each chunk and each warp
+// releases a chunk when its lanes are done with it.
+//
+// stream_chunks streams chunks chunk_of(0), ..., chunk_of(n - 1) and calls
+// f(full, a, ia, b, ib, va, vb) for each: a and b the thread's two float4s,
+// ia and ib their float4 indices in the row, va and vb whether they lie in the
+// row, and `full` (a type) true at compile time for every chunk but a partial
+// last one. sm.ring_q[t] counts the chunks the CTA has consumed so far (the
+// same on every thread); it fixes the parity of every ring barrier. Returns
+// false when a bounded wait gave up: sm.abort_flag is then raised,
+// STS_ERR_TIMEOUT recorded in *sm.err, and thread 0 has waited (bounded) for
+// its copies in flight.
+template <typename CF, typename F>
+__device__ __forceinline__ bool stream_chunks(RSmem& sm, const float4* __restrict__ x4, int V4,
+                                              int n, CF&& chunk_of, unsigned long long policy,
+                                              F&& f) {
+  int* err = sm.err;
+  const int tid = (int)threadIdx.x, lane = tid & 31;
+  volatile int* abort_flag = &sm.abort_flag;
+  const uint32_t q0 = sm.ring_q[tid];
+  int issued = 0;  // thread 0
+  auto issue = [&](int j) -> bool {
+    const uint32_t qq = q0 + (uint32_t)j;
+    const int s = (int)(qq % NSTAGE);
+    if (qq >= (uint32_t)NSTAGE &&
+        !mbar_wait(smem_u32(&sm.empty_bar[s]), ((qq / NSTAGE) - 1u) & 1u, abort_flag, err))
+      return false;
+    const int f0 = chunk_of(j) * CH_F4;
+    const uint32_t bytes = (uint32_t)min(CH_F4, V4 - f0) * 16u;
+    mbar_arrive_expect_tx(smem_u32(&sm.full_bar[s]), bytes);
+    bulk_load(smem_u32(&sm.ring[s][0]), x4 + f0, bytes, smem_u32(&sm.full_bar[s]), policy);
+    ++issued;
+    return true;
+  };
+  bool ok = true;
+  if (tid == 0)
+    for (int j = 0; j < n && j < NSTAGE && ok; ++j) ok = issue(j);
+  int j = 0;
+  for (; j < n && ok; ++j) {
+    const uint32_t qq = q0 + (uint32_t)j;
+    const int s = (int)(qq % NSTAGE);
+    if (!mbar_wait(smem_u32(&sm.full_bar[s]), (qq / NSTAGE) & 1u, abort_flag, err)) {
+      ok = false;
+      break;
+    }
+    const int f0 = chunk_of(j) * CH_F4;
+    const int cnt = min(CH_F4, V4 - f0);
+    const float4 a = sm.ring[s][tid];
+    const float4 b = sm.ring[s][tid + RT];
+    if (cnt == CH_F4)
+      f(std::true_type{}, a, f0 + tid, b, f0 + tid + RT, true, true);
+    else
+      f(std::false_type{}, a, f0 + tid, b, f0 + tid + RT, tid < cnt, tid + RT < cnt);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&sm.empty_bar[s]));
+    if (tid == 0 && j + NSTAGE < n && ok) ok = issue(j + NSTAGE);
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    if (tid == 0)  // copies issued but not consumed may still be landing
+      for (int k = j; k < issued; ++k) {
+        const uint32_t qq = q0 + (uint32_t)k;
+        mbar_wait_drain(smem_u32(&sm.full_bar[qq % NSTAGE]), (qq / NSTAGE) & 1u);
+      }
+  }
+  sm.ring_q[tid] = q0 + (uint32_t)n;
+  return ok;
+}
+
+// Number of chunks of a row of V4 float4s.
+__device__ __forceinline__ int n_chunks(int V4) { return (V4 + CH_F4 - 1) / CH_F4; }
 
 // ---------------------------------------------------------------- block reductions
 // Fixed shuffle-down trees: results are identical on every run.
@@ -426,10 +525,13 @@ __device__ void block_exscan_d3(const double (&v)[3], double (&pre)[3], double (
 
 enum Crit : int { kCount = 0, kMassGE = 1, kMassGT = 2 };
 
+constexpr double kNoQx = __builtin_nan("");
+
 struct Cut {
   unsigned long long K;  // composite key of the last element of the prefix
   long long cnt;         // prefix length
   double mass;           // prefix mass sum exp(s - m)
+  double qx = kNoQx;     // prefix sum of exp(s - m) (s - m), when the path formed it
 };
 
 __device__ __forceinline__ bool crit_ok(int crit, long long c, double mss, long long need, double target) {
@@ -851,12 +953,60 @@ __device__ __noinline__ bool resolve_row_exact(RSmem& sm, const float* __restric
 
 // ---------------------------------------------------------------- fast path
 
-// Count-only level-0 histogram.
+// Whether element e belongs to the planning sample (with float4 streaming, one
+// chunk in SAMPLE_EVERY and the scalar tail; else one block of RT elements in
+// SAMPLE_EVERY): see sample_hist.
 template <bool VEC>
-__device__ __noinline__ void count_hist(RSmem& sm, const float* __restrict__ x, int V, float m) {
-  for (int i = threadIdx.x; i < NB; i += RT) sm.cnt[i] = 0;
-  __syncthreads();
-  for_each<VEC, true>(x, V, [&](float s, int) { atomicAdd(&sm.cnt[bin0(s, m)], 1); });
+__device__ __forceinline__ bool in_sample(int e, int V) {
+  if (VEC) return e >= (V & ~3) || (((e >> 2) / CH_F4) % SAMPLE_EVERY) == 0;
+  return ((e / RT) % SAMPLE_EVERY) == 0;
+}
+
+// Count-only level-0 histogram. With `sampled`, sm.cnt already holds the
+// counts of the planning sample and only the other elements are added.
+template <bool VEC>
+__device__ __noinline__ void count_hist(RSmem& sm, const float* __restrict__ x, int V, float m,
+                                        bool sampled) {
+  if (!sampled) {
+    for (int i = threadIdx.x; i < NB; i += RT) sm.cnt[i] = 0;
+    __syncthreads();
+  }
+  if (VEC) {
+    // every chunk, or the ones the sample skipped (chunk j + j / 7 + 1 is the
+    // j-th chunk that is not a multiple of SAMPLE_EVERY)
+    const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
+    const int V4 = V >> 2;
+    const int nch = n_chunks(V4);
+    const int n = sampled ? nch - (nch + SAMPLE_EVERY - 1) / SAMPLE_EVERY : nch;
+    auto body = [&](auto, const float4& u, int, const float4& w, int, bool vu, bool vw) {
+      if (vu) {
+        atomicAdd(&sm.cnt[bin0(u.x, m)], 1);
+        atomicAdd(&sm.cnt[bin0(u.y, m)], 1);
+        atomicAdd(&sm.cnt[bin0(u.z, m)], 1);
+        atomicAdd(&sm.cnt[bin0(u.w, m)], 1);
+      }
+      if (vw) {
+        atomicAdd(&sm.cnt[bin0(w.x, m)], 1);
+        atomicAdd(&sm.cnt[bin0(w.y, m)], 1);
+        atomicAdd(&sm.cnt[bin0(w.z, m)], 1);
+        atomicAdd(&sm.cnt[bin0(w.w, m)], 1);
+      }
+    };
+    if (sampled)
+      stream_chunks(sm, x4, V4, n,
+                    [](int j) { return j + j / (SAMPLE_EVERY - 1) + 1; }, l2_policy_keep(), body);
+    else
+      stream_chunks(sm, x4, V4, n, [](int j) { return j; }, l2_policy_keep(), body);
+    if (!sampled)
+      for (int i = 4 * V4 + (int)threadIdx.x; i < V; i += RT)
+        atomicAdd(&sm.cnt[bin0(ld_stream(x + i), m)], 1);
+  } else if (!sampled) {
+    for_each<false, true>(x, V, [&](float s, int) { atomicAdd(&sm.cnt[bin0(s, m)], 1); });
+  } else {
+    for_each<false, true>(x, V, [&](float s, int e) {
+      if (!in_sample<false>(e, V)) atomicAdd(&sm.cnt[bin0(s, m)], 1);
+    });
+  }
   __syncthreads();
 }
 
@@ -867,19 +1017,13 @@ __device__ long long count_range(RSmem& sm, int lo, int hi) {
   return block_sum_l(c, sm);
 }
 
+// Results of pass 2.
 struct Pass2 {
-  // plan
-  bool need_z;       // exact total mass (and mass before w_lo / b_mu) for every element
-  bool need_last;    // last element of the order
-  int w_lo, w_hi;    // window of buckets gathered by bucket into regions (w_lo > w_hi: none)
-  int woff[3];       // region offsets in sm.cand of the window buckets
-  int b_mu;          // min-p boundary bucket (-1: min-p off)
-  uint32_t kt;       // min-p threshold key
-  int bk;            // gather every bucket <= bk into sm.cand (-1: no prefix gather)
-  // results
-  double z, a_p, a_mu;
-  unsigned long long k_last;
-  bool overflow;     // a warp's gather slice overflowed
+  double z, a_p, a_mu;       // total mass, mass before w_lo, mass before b_mu
+  double zx, a_px, a_mux;    // the same sums of exp(s - m) (s - m) (when asked)
+  long long c_p, c_mu;       // counts before w_lo and before b_mu (when counted)
+  unsigned long long k_last; // last element of the order (when asked)
+  bool overflow;             // a warp's gather slice overflowed
 };
 
 // Plan of pass 2, passed by value so every field lives in a register.
@@ -889,6 +1033,7 @@ struct Plan2 {
   int g2_lo, g2_hi;         // ... and [g2_lo, g2_hi] (empty ranges: lo > hi)
   int w_lo;                 // mass before w_lo is accumulated (a_p)
   int b_mu;                 // mass before b_mu is accumulated (a_mu); -1: off
+  int ent;                  // also sum exp(s - m) (s - m) per region (entropy)
 };
 
 constexpr int WCAP = CAP / NWARP;  // private gather slots per warp
@@ -900,7 +1045,7 @@ constexpr int WCAP = CAP / NWARP;  // private gather slots per warp
 // chains and summed into split accumulators, so float64 latency is covered.
 // Every lane of a warp runs every batch (invalid slots masked), so the warp
 // votes always see the full warp.
-template <bool VEC, bool NEED_Z>
+template <bool VEC, bool NEED_Z, bool COUNTS>
 __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, int V, float m,
                                         const Plan2 pl, Pass2& P) {
   constexpr int E = 8;
@@ -909,10 +1054,18 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
   const int g_lo = pl.g_lo, g_hi = pl.g_hi, g2_lo = pl.g2_lo, g2_hi = pl.g2_hi;
   const int w_lo = pl.w_lo, b_mu = pl.b_mu;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
+  // gather ranges as (start, span) for one unsigned compare each; an empty
+  // range (lo > hi) gets a start no bucket reaches
+  const unsigned g1s = g_lo <= g_hi ? (unsigned)g_lo : 0x80000000u;
+  const unsigned g1n = g_lo <= g_hi ? (unsigned)(g_hi - g_lo) : 0u;
+  const unsigned g2s = g2_lo <= g2_hi ? (unsigned)g2_lo : 0x80000000u;
+  const unsigned g2n = g2_lo <= g2_hi ? (unsigned)(g2_hi - g2_lo) : 0u;
   unsigned long long* wbuf = sm.cand + warp * WCAP;
   int wfill = 0;  // warp-uniform
   double z[2] = {0.0, 0.0}, ap[2] = {0.0, 0.0}, amu[2] = {0.0, 0.0};
+  double zx = 0.0, apx = 0.0, amux = 0.0;  // the same sums of q (s - m) (entropy)
+  const bool ent = pl.ent != 0;
+  int cp = 0, cmu = 0;  // counts before w_lo and before b_mu (COUNTS)
   unsigned long long kl = ~0ull;
 
   // Element e < 4 of a batch is token a0 + e (valid when e < na), element
@@ -955,15 +1108,35 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
       }
 #pragma unroll
       for (int e = 0; e < E; ++e) qq[e] = ok(e) ? qq[e] : 0.0;
+      // predicated adds (no selects): a region's sum only takes its elements
       if (NEED_Z)
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           z[e & 1] += qq[e];
-          ap[e & 1] += bb[e] < w_lo ? qq[e] : 0.0;
+          if (bb[e] < w_lo) ap[e & 1] += qq[e];
         }
       if (need_mu)
 #pragma unroll
-        for (int e = 0; e < E; ++e) amu[e & 1] += bb[e] < b_mu ? qq[e] : 0.0;
+        for (int e = 0; e < E; ++e)
+          if (bb[e] < b_mu) amu[e & 1] += qq[e];
+      if (ent) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const double qx = ok(e) ? qq[e] * ((double)sv[e] - md) : 0.0;
+          if (NEED_Z) {
+            zx += qx;
+            if (bb[e] < w_lo) apx += qx;
+          }
+          if (need_mu && bb[e] < b_mu) amux += qx;
+        }
+      }
+    }
+    if (COUNTS) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        if (ok(e) && bb[e] < w_lo) ++cp;
+        if (ok(e) && bb[e] < b_mu) ++cmu;
+      }
     }
     if (need_last) {
 #pragma unroll
@@ -975,52 +1148,44 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
     unsigned gm = 0;  // this thread's elements in a gathered range, one bit each
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      const int b = bb[e];
-      const bool g = ok(e) && ((b >= g_lo && b <= g_hi) || (b >= g2_lo && b <= g2_hi));
+      const unsigned b = (unsigned)bb[e];
+      const bool g = ok(e) && (b - g1s <= g1n || b - g2s <= g2n);
       gm |= g ? 1u << e : 0u;
     }
+    // One slot range per thread from a warp scan of its hit count (hits are
+    // rare: a vote skips batches without any), then the hits stored in order.
     if (__any_sync(0xffffffffu, gm != 0u)) {
+      const int c = __popc(gm);
+      int incl = c;
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const bool g = (gm >> e) & 1u;
-        const unsigned mk = __ballot_sync(0xffffffffu, g);
-        const int slot = wfill + __popc(mk & lt);
-        if (g && slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
-        wfill += __popc(mk);
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
+      int slot = wfill + incl - c;
+      wfill += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if ((gm >> e) & 1u) {
+          if (slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
+          ++slot;
+        }
     }
   };
 
   const int tid = (int)threadIdx.x;
   int tail0 = 0;  // first token handled one per thread
   if (VEC) {
-    // Fully coalesced: in each sweep thread t reads float4s base + u * RT + t
-    // (u = 0..3), so every warp load covers 512 contiguous bytes; a batch
-    // pairs two of those float4s.
+    // the row streams through the ring; a batch is the thread's two float4s
+    // of a chunk (the loads read evict-first: this is the row's last pass)
     const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
     const int V4 = V >> 2;
-    const unsigned long long drop = l2_policy_drop();
-    const int full_end = V4 - V4 % (RT * 4);  // sweeps where every thread's loads are in the row
-    for (int base = 0; base < full_end; base += RT * 4) {
-      float4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = ld_stream4(x4 + base + u * RT + tid, drop);
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int ia = base + 2 * h * RT + tid, ib = ia + RT;
-        const float4 a4 = h ? v[2] : v[0], b4 = h ? v[3] : v[1];
-        const float sv[E] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
-        batch(std::true_type{}, sv, 4 * ia, 4, 4 * ib, 4);
-      }
-    }
-    for (int base = full_end; base < V4; base += RT * 2) {  // the last partial sweep
-      const int ia = base + tid, ib = ia + RT;
-      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 a4 = ia < V4 ? ld_stream4(x4 + ia, drop) : z4;
-      const float4 b4 = ib < V4 ? ld_stream4(x4 + ib, drop) : z4;
-      const float sv[E] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
-      batch(std::false_type{}, sv, 4 * ia, ia < V4 ? 4 : 0, 4 * ib, ib < V4 ? 4 : 0);
-    }
+    stream_chunks(sm, x4, V4, n_chunks(V4), [](int j) { return j; }, l2_policy_drop(),
+                  [&](auto full, const float4& a4, int ia, const float4& b4, int ib, bool va,
+                      bool vb) {
+                    const float sv[E] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+                    batch(full, sv, 4 * ia, va ? 4 : 0, 4 * ib, vb ? 4 : 0);
+                  });
     tail0 = 4 * V4;
   }
   for (int i0 = tail0; i0 < V; i0 += RT) {
@@ -1031,11 +1196,19 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
     batch(std::false_type{}, sv, i, in ? 1 : 0, i, 0);
   }
   if (lane == 0) sm.wcount[warp] = wfill;
-  double sums[3] = {z[0] + z[1], ap[0] + ap[1], amu[0] + amu[1]};
-  block_sum_multi<3>(sums, sm);
-  P.z = sums[0];
-  P.a_p = sums[1];
-  P.a_mu = sums[2];
+  {
+    double sums[8] = {z[0] + z[1], ap[0] + ap[1], amu[0] + amu[1], (double)cp, (double)cmu,
+                      zx, apx, amux};
+    block_sum_multi<8>(sums, sm);  // counts are exact in a double
+    P.z = sums[0];
+    P.a_p = sums[1];
+    P.a_mu = sums[2];
+    P.c_p = (long long)sums[3];
+    P.c_mu = (long long)sums[4];
+    P.zx = sums[5];
+    P.a_px = sums[6];
+    P.a_mux = sums[7];
+  }
   P.k_last = need_last ? block_ext_u<false>(kl, sm) : ~0ull;
   int ovf = 0;
   for (int w = 0; w < NWARP; ++w) ovf |= sm.wcount[w] > WCAP ? 1 : 0;
@@ -1045,11 +1218,163 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
 
 template <bool VEC>
 __device__ void pass2(RSmem& sm, const float* __restrict__ x, int V, float m, bool need_z,
-                      const Plan2& pl, Pass2& P) {
-  if (need_z)
-    pass2_impl<VEC, true>(sm, x, V, m, pl, P);
-  else
-    pass2_impl<VEC, false>(sm, x, V, m, pl, P);
+                      const Plan2& pl, Pass2& P, bool counts = false) {
+  if (counts) {
+    if (need_z)
+      pass2_impl<VEC, true, true>(sm, x, V, m, pl, P);
+    else
+      pass2_impl<VEC, false, true>(sm, x, V, m, pl, P);
+  } else {
+    if (need_z)
+      pass2_impl<VEC, true, false>(sm, x, V, m, pl, P);
+    else
+      pass2_impl<VEC, false, false>(sm, x, V, m, pl, P);
+  }
+}
+
+// ---------------------------------------------------------------- min-p pass
+// One pass for a row whose min-p prefix decides the support. Elements in
+// buckets below g_lo are all kept: their values are compacted per warp into a
+// staging area and weighed in float64 in full batches (so the float64 work
+// follows the kept elements, not the row). Elements in buckets [g_lo, g_hi]
+// are gathered (their keys decide which are kept). Elements after g_hi are
+// dropped: they only add tab[b] per element to a lower bound of their mass,
+// exact since each weighs at least tab[b] exp(-1/128) and at most tab[b].
+struct MuPass {
+  double mass, qx;     // kept elements before g_lo: mass and sum of q (s - m)
+  long long cnt;       // their number
+  double rest_upper;   // sum of tab[b] over the elements after g_hi
+  bool overflow;       // a gather slice or the staging area overflowed
+};
+
+constexpr int MU_STAGE = 512;  // staged values per warp (the storage of sm.mass)
+static_assert(NWARP * MU_STAGE * 4 <= NB * 8, "the staging area fits the bucket-mass storage");
+
+template <bool VEC>
+__device__ __noinline__ void mu_pass(RSmem& sm, const float* __restrict__ x, int V, float m,
+                                     int g_lo, int g_hi, bool ent, MuPass& out) {
+  constexpr int E = 8;
+  const double md = (double)m;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* stage = reinterpret_cast<float*>(sm.mass) + warp * MU_STAGE;
+  unsigned long long* wbuf = sm.cand + warp * WCAP;
+  int sfill = 0, wfill = 0;  // warp-uniform fill levels
+  double mass = 0.0, qx = 0.0, rest = 0.0;
+  int cnt = 0;
+  const unsigned gs = (unsigned)g_lo, gn = (unsigned)(g_hi - g_lo);
+
+  // weigh `n` staged values (n <= 8 * 32, lane j takes j, j + 32, ...)
+  auto weigh = [&](int n) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int i = e * 32 + lane;
+      if (i < n) {
+        const float s = stage[i];
+        const int b = bin0(s, m);
+        const double q = qmass_b(sm.tab, s, md, b);
+        mass += q;
+        if (ent) qx += q * ((double)s - md);
+      }
+    }
+  };
+
+  auto batch = [&](auto full, const float (&sv)[E], int a0, int na, int b0, int nb) {
+    auto idx = [&](int e) { return e < 4 ? a0 + e : b0 + (e - 4); };
+    auto ok = [&](int e) { return decltype(full)::value || (e < 4 ? e < na : e - 4 < nb); };
+    unsigned pre = 0, gm = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int b = bin0(sv[e], m);
+      const bool v = ok(e);
+      pre |= (v && b < g_lo) ? 1u << e : 0u;
+      gm |= (v && (unsigned)b - gs <= gn) ? 1u << e : 0u;
+      if (v && b > g_hi) rest += tab_at(sm.tab, b);
+    }
+    cnt += __popc(pre);
+    // stage the kept values: one slot range per thread from a warp scan
+    {
+      const int c = __popc(pre);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int slot = sfill + incl - c;
+      sfill += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if ((pre >> e) & 1u) stage[slot++] = sv[e];
+      __syncwarp();
+      if (sfill >= 8 * 32) {  // a full batch: weigh it, move the rest to the front
+        weigh(8 * 32);
+        const int left = sfill - 8 * 32;  // < 8 * 32
+        float keep[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = e * 32 + lane;
+          keep[e] = i < left ? stage[8 * 32 + i] : 0.f;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = e * 32 + lane;
+          if (i < left) stage[i] = keep[e];
+        }
+        __syncwarp();
+        sfill = left;
+      }
+    }
+    if (__any_sync(0xffffffffu, gm != 0u)) {
+      const int c = __popc(gm);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int slot = wfill + incl - c;
+      wfill += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if ((gm >> e) & 1u) {
+          if (slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
+          ++slot;
+        }
+    }
+  };
+
+  const int tid = (int)threadIdx.x;
+  int tail0 = 0;
+  if (VEC) {
+    const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
+    const int V4 = V >> 2;
+    stream_chunks(sm, x4, V4, n_chunks(V4), [](int j) { return j; }, l2_policy_drop(),
+                  [&](auto full, const float4& a4, int ia, const float4& b4, int ib, bool va,
+                      bool vb) {
+                    const float sv[E] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+                    batch(full, sv, 4 * ia, va ? 4 : 0, 4 * ib, vb ? 4 : 0);
+                  });
+    tail0 = 4 * V4;
+  }
+  for (int i0 = tail0; i0 < V; i0 += RT * 2) {
+    const int ia = i0 + tid, ib = ia + RT;
+    const float a = ia < V ? ld_stream(x + ia) : 0.f, b = ib < V ? ld_stream(x + ib) : 0.f;
+    const float sv[E] = {a, a, a, a, b, b, b, b};
+    batch(std::false_type{}, sv, ia, ia < V ? 1 : 0, ib, ib < V ? 1 : 0);
+  }
+  weigh(sfill);  // the last partial batch
+  if (lane == 0) sm.wcount[warp] = wfill;
+  double sums[4] = {mass, qx, rest, (double)cnt};  // counts are exact in a double
+  block_sum_multi<4>(sums, sm);
+  out.mass = sums[0];
+  out.qx = sums[1];
+  out.rest_upper = sums[2];
+  out.cnt = (long long)sums[3];
+  int ovf = 0;
+  for (int w = 0; w < NWARP; ++w) ovf |= sm.wcount[w] > WCAP ? 1 : 0;
+  out.overflow = ovf != 0;
+  __syncthreads();
 }
 
 // Packs the live keys of the per-warp slices densely, in slice order, into the
@@ -1102,9 +1427,10 @@ __device__ __noinline__ int compact_gathered(RSmem& sm, int n, float m, int lo, 
 // min-p) of those with key >= kt, plus the smallest such key.
 __device__ __noinline__ void gathered_bucket_stats(RSmem& sm, int n, float m, int b, uint32_t kt,
                                                    double& mass, long long& cnt, double& kept_mass,
-                                                   long long& kept_cnt, unsigned long long& k_min) {
+                                                   long long& kept_cnt, unsigned long long& k_min,
+                                                   double& kept_qx) {
   const unsigned long long* g = packed(sm);
-  double ms = 0.0, km = 0.0;
+  double ms = 0.0, km = 0.0, kx = 0.0;
   long long c = 0, kc = 0;
   unsigned long long kmn = ~0ull;
   for (int i = threadIdx.x; i < n; i += RT) {
@@ -1116,44 +1442,61 @@ __device__ __noinline__ void gathered_bucket_stats(RSmem& sm, int n, float m, in
     ++c;
     if ((uint32_t)(K >> 32) >= kt) {
       km += q;
+      kx += q * ((double)v - (double)m);
       ++kc;
       kmn = K < kmn ? K : kmn;
     }
   }
-  double v[4] = {ms, (double)c, km, (double)kc};  // counts are exact in a double
-  block_sum_multi<4>(v, sm);
+  double v[5] = {ms, (double)c, km, (double)kc, kx};  // counts are exact in a double
+  block_sum_multi<5>(v, sm);
   mass = v[0];
   cnt = (long long)v[1];
   kept_mass = v[2];
   kept_cnt = (long long)v[3];
+  kept_qx = v[4];
   k_min = block_ext_u<false>(kmn, sm);
 }
 
 // Exact masses and counts of the n packed candidates of buckets lo..hi
 // (hi - lo <= 2).
 __device__ __noinline__ void window_stats(RSmem& sm, int n, float m, int lo, int hi,
-                                          double (&wm)[3], long long (&wc)[3]) {
+                                          double (&wm)[3], long long (&wc)[3], double (&wqx)[3]) {
   const unsigned long long* g = packed(sm);
-  double ms[3] = {0.0, 0.0, 0.0};
+  double ms[3] = {0.0, 0.0, 0.0}, mx[3] = {0.0, 0.0, 0.0};
   long long c[3] = {0, 0, 0};
   for (int i = threadIdx.x; i < n; i += RT) {
     const float v = ckey_value(g[i]);
     const int w = bin0(v, m) - lo;
     if (w < 0 || w > hi - lo) continue;
     const double q = qmass(sm, v, m);
+    const double qx = q * ((double)v - (double)m);
 #pragma unroll
     for (int u = 0; u < 3; ++u) {
       ms[u] += w == u ? q : 0.0;
+      mx[u] += w == u ? qx : 0.0;
       c[u] += w == u ? 1 : 0;
     }
   }
   double v[6] = {ms[0], ms[1], ms[2], (double)c[0], (double)c[1], (double)c[2]};
   block_sum_multi<6>(v, sm);
+  block_sum_multi<3>(mx, sm);
 #pragma unroll
   for (int w = 0; w < 3; ++w) {
     wm[w] = v[w];
     wc[w] = (long long)v[3 + w];
+    wqx[w] = mx[w];
   }
+}
+
+// Sum of exp(s - m) (s - m) over the first n keys of sm.cand (sorted): the
+// part of the support's entropy sum that lies among the sorted candidates.
+__device__ __noinline__ double sorted_prefix_qx(RSmem& sm, int n, float m) {
+  double acc = 0.0;
+  for (int j = threadIdx.x; j < n; j += RT) {
+    const float v = ckey_value(sm.cand[j]);
+    acc += qmass(sm, v, m) * ((double)v - (double)m);
+  }
+  return block_sum_d(acc, sm);
 }
 
 // Last non-empty bucket strictly before b (-1 if none).
@@ -1237,11 +1580,72 @@ __device__ __noinline__ TopPPlan plan_top_p(RSmem& sm, float p) {
   return pl;
 }
 
+// Top-k whose prefix up to the k-th element's bucket holds more than SCAP
+// elements. The exact counts place the k-th element in bucket bk (with ce
+// elements before it); one exact pass weighs everything before bk and gathers
+// bk alone, whose sorted elements give the k-th element and the top-k mass
+// Z_k = (mass before bk) + (prefix of bk). Min-p cuts earlier than the k-th
+// element only when its threshold's bucket bm <= bk: within bk it is read off
+// the sorted bucket, before bk one pass counts its prefix. With top-p, the
+// crossing on the top-k-renormalised mass (target p Z_k, known only now) is
+// placed by the exact search's locate. Returns false when bucket bk alone
+// exceeds the sort (the exact search then decides).
+template <bool VEC>
+__device__ __noinline__ bool resolve_large_k(RSmem& sm, const float* __restrict__ x, int V, float m,
+                                             int k, float p, float mu, uint32_t kt, bool ent,
+                                             int bk, long long ce, Cut& best) {
+  const bool p_on = p < 1.0f, mu_on = mu > 0.0f;
+  if (sm.cnt[bk] > SCAP) return false;
+  Plan2 pl;
+  pl.need_last = 0;
+  pl.g_lo = bk;
+  pl.g_hi = bk;
+  pl.g2_lo = 1;
+  pl.g2_hi = 0;
+  pl.w_lo = bk;  // a_p: the mass before bk
+  pl.b_mu = -1;
+  pl.ent = ent ? 1 : 0;
+  Pass2 P;
+  pass2<VEC>(sm, x, V, m, true, pl, P);
+  if (P.overflow) return false;
+  const int ng = pack_gathered(sm);
+  const int n = compact_gathered(sm, ng, m, bk, bk);
+  const int jk = (int)((long long)k - ce) - 1;
+  if (jk < 0 || jk >= n) return false;
+  sort_and_scan(sm, n, m);
+  best = Cut{sm.cand[jk], (long long)k, P.a_p + sm.cq[jk]};
+  const double Zk = best.mass;
+  if (mu_on) {
+    const int bm = bin0(key32_value(kt), m);
+    if (bm == bk) {
+      int mine = 0;
+      for (int j = threadIdx.x; j < n; j += RT) mine += (uint32_t)(sm.cand[j] >> 32) >= kt ? 1 : 0;
+      const int nk = (int)block_sum_l(mine, sm);  // kept elements of bk: a prefix of it
+      if (nk >= 1)
+        take_earlier(best, Cut{sm.cand[nk - 1], ce + nk, P.a_p + sm.cq[nk - 1]});
+      else  // nothing of bk kept: the min-p prefix ends in an earlier bucket
+        take_earlier(best, min_p_cut_pass<VEC>(sm, x, V, m, kt));
+    } else if (bm < bk) {
+      take_earlier(best, min_p_cut_pass<VEC>(sm, x, V, m, kt));
+    }
+  }
+  if (ent && best.cnt > ce) best.qx = P.a_px + sorted_prefix_qx(sm, (int)(best.cnt - ce), m);
+  if (p_on) {
+    bool hist_valid = false;
+    Cut cp;
+    if (!locate<VEC>(sm, x, V, m, hist_valid, kMassGE, 0, (double)p * Zk, cp)) return false;
+    take_earlier(best, cp);
+  }
+  __syncthreads();
+  return true;
+}
+
 // Resolve a row with one count pass and one exact pass. Returns false when the
 // exact path must decide instead.
 template <bool VEC>
 __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict__ x, int V, float m,
-                                              int k, float p, float mu, uint32_t kt, Cut& best) {
+                                              int k, float p, float mu, uint32_t kt, bool sampled,
+                                              bool ent, Cut& best) {
   const bool k_on = k >= 1 && k < V, p_on = p < 1.0f, mu_on = mu > 0.0f;
   Plan2 pl;
   pl.need_last = 0;
@@ -1251,16 +1655,17 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
   pl.g2_hi = 0;
   pl.w_lo = -1;
   pl.b_mu = -1;
+  pl.ent = ent ? 1 : 0;
   Pass2 P;
 
   if (!k_on && !p_on && !mu_on) {  // identity: total mass and the last element only
     pl.need_last = 1;
     pass2<VEC>(sm, x, V, m, true, pl, P);
-    best = Cut{P.k_last, (long long)V, P.z};
+    best = Cut{P.k_last, (long long)V, P.z, P.zx};
     return true;
   }
 
-  count_hist<VEC>(sm, x, V, m);
+  count_hist<VEC>(sm, x, V, m, sampled);
 
   if (k_on) {
     // small k: the prefix of buckets up to the k-th element's fits the buffer
@@ -1271,7 +1676,7 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
     pick_bucket(sm, kCount, (long long)k, 0.0, 0, 0.0, bk, ce, me);
     const long long incl = ce + sm.cnt[bk];
     __syncthreads();
-    if (incl > SCAP) return false;  // keep the per-warp slices far from full
+    if (incl > SCAP) return resolve_large_k<VEC>(sm, x, V, m, k, p, mu, kt, ent, bk, ce, best);
     pl.g_lo = 0;
     pl.g_hi = bk;
     pass2<VEC>(sm, x, V, m, false, pl, P);
@@ -1293,6 +1698,7 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
       const int nk = (int)block_sum_l(mine, sm);
       if (nk >= 1 && nk < n) take_earlier(best, Cut{sm.cand[nk - 1], (long long)nk, sm.cq[nk - 1]});
     }
+    if (ent) best.qx = sorted_prefix_qx(sm, (int)best.cnt, m);  // the support is a sorted prefix
     __syncthreads();
     return true;
   }
@@ -1342,26 +1748,26 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
 
     bool have = false;
     if (mu_on) {
-      double mass, kmass;
+      double mass, kmass, kqx;
       long long cnt, kcnt;
       unsigned long long kmin;
-      gathered_bucket_stats(sm, ng, m, bm, kt, mass, cnt, kmass, kcnt, kmin);
+      gathered_bucket_stats(sm, ng, m, bm, kt, mass, cnt, kmass, kcnt, kmin, kqx);
       if (kcnt == 0 && bprev >= 0) {
         // nothing of bucket bm is kept: the min-p prefix ends with bucket bprev
-        double m2, k2;
+        double m2, k2, x2;
         long long c2, kc2;
-        gathered_bucket_stats(sm, ng, m, bprev, 0u, m2, c2, k2, kc2, kmin);
+        gathered_bucket_stats(sm, ng, m, bprev, 0u, m2, c2, k2, kc2, kmin, x2);
       }
-      best = Cut{kmin, before_mu + kcnt, P.a_mu + kmass};
+      best = Cut{kmin, before_mu + kcnt, P.a_mu + kmass, P.a_mux + kqx};
       have = true;
     }
     if (p_on) {
       const double target = (double)p * P.z;
       // the crossing bucket, from the exact masses of the gathered window
-      double wm[3];
+      double wm[3], wqx[3];
       long long wc[3];
-      window_stats(sm, ng, m, lo, hi, wm, wc);
-      double before = P.a_p;
+      window_stats(sm, ng, m, lo, hi, wm, wc, wqx);
+      double before = P.a_p, before_qx = P.a_px;
       long long cbefore = before_win;
       int c = -1;
       for (int w = lo; w <= hi; ++w) {
@@ -1370,6 +1776,7 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
           break;
         }
         before += wm[w - lo];
+        before_qx += wqx[w - lo];
         cbefore += wc[w - lo];
       }
       if (c < 0) {  // the crossing lies outside the window
@@ -1379,7 +1786,8 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
       const int n = compact_gathered(sm, ng, m, c, c);
       sort_and_scan(sm, n, m);
       const int jp = first_mass_hit(sm, 0, n, before, 0.0, kMassGE, target);
-      const Cut cp{sm.cand[jp], cbefore + jp + 1, before + sm.cq[jp]};
+      const double qx = ent ? before_qx + sorted_prefix_qx(sm, jp + 1, m) : kNoQx;
+      const Cut cp{sm.cand[jp], cbefore + jp + 1, before + sm.cq[jp], qx};
       if (have)
         take_earlier(best, cp);
       else
@@ -1391,13 +1799,281 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
   return false;
 }
 
+// Sum of exp(s - m) (s - m) over the support (every element whose composite
+// key is >= K, the key of its last element): one pass over the row, for rows
+// decided by the exact search, whose histograms carry masses only.
+template <bool VEC>
+__device__ __noinline__ double support_qx_pass(RSmem& sm, const float* __restrict__ x, int V,
+                                               float m, unsigned long long K) {
+  double acc = 0.0;
+  for_each<VEC>(x, V, [&](float s, int i) {
+    if (ckey(s, i) >= K) acc += qmass(sm, s, m) * ((double)s - (double)m);
+  });
+  return block_sum_d(acc, sm);
+}
+
+// ---------------------------------------------------------------- planned path
+// The first attempt for every filtered row. A sample of the row (one sweep in
+// SAMPLE_EVERY) feeds a count histogram from which the gathered range is
+// planned: for top-k the buckets up to the k-th element, for min-p the
+// buckets around its threshold (when top-p is on too, only if the sample puts
+// the top-p crossing clearly after the min-p prefix). One pass then gathers
+// that range and, for min-p, counts and weighs everything before it (float64
+// masses, exact counts), and the row is decided from those. A plan the pass
+// does not confirm (fewer than k elements gathered, a buffer too small, top-p
+// deciding after all), and every row whose top-p crossing decides, goes to
+// the fast path above, whose count pass adds the rest of the row to the
+// sample's counts, and from there to the exact search: the result never
+// rests on the sample, only the amount of work does.
+
+// Count histogram of the planning sample in sm.cnt. Returns the sample size.
+template <bool VEC>
+__device__ __noinline__ int sample_hist(RSmem& sm, const float* __restrict__ x, int V, float m) {
+  for (int i = threadIdx.x; i < NB; i += RT) sm.cnt[i] = 0;
+  __syncthreads();
+  const int tid = (int)threadIdx.x;
+  int n = 0;  // uniform over the block
+  if (VEC) {
+    // chunks 0, SAMPLE_EVERY, 2 SAMPLE_EVERY, ... and the scalar tail
+    const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
+    const int V4 = V >> 2;
+    const int nch = n_chunks(V4);
+    const int ns = (nch + SAMPLE_EVERY - 1) / SAMPLE_EVERY;
+    stream_chunks(sm, x4, V4, ns, [](int j) { return j * SAMPLE_EVERY; }, l2_policy_keep(),
+                  [&](auto, const float4& u, int, const float4& w, int, bool vu, bool vw) {
+                    if (vu) {
+                      atomicAdd(&sm.cnt[bin0(u.x, m)], 1);
+                      atomicAdd(&sm.cnt[bin0(u.y, m)], 1);
+                      atomicAdd(&sm.cnt[bin0(u.z, m)], 1);
+                      atomicAdd(&sm.cnt[bin0(u.w, m)], 1);
+                    }
+                    if (vw) {
+                      atomicAdd(&sm.cnt[bin0(w.x, m)], 1);
+                      atomicAdd(&sm.cnt[bin0(w.y, m)], 1);
+                      atomicAdd(&sm.cnt[bin0(w.z, m)], 1);
+                      atomicAdd(&sm.cnt[bin0(w.w, m)], 1);
+                    }
+                  });
+    for (int j = 0; j < ns; ++j) n += 4 * min(CH_F4, V4 - j * SAMPLE_EVERY * CH_F4);
+    for (int i = 4 * V4 + tid; i < V; i += RT) atomicAdd(&sm.cnt[bin0(ld_stream(x + i), m)], 1);
+    n += V - 4 * V4;  // the scalar tail (< 4 elements) is always in the sample
+  } else {
+    for (int base = 0; base < V; base += RT * SAMPLE_EVERY) {
+      const int i = base + tid;
+      if (i < V) atomicAdd(&sm.cnt[bin0(ld_stream(x + i), m)], 1);
+      n += min(RT, V - base);
+    }
+  }
+  __syncthreads();
+  return n;
+}
+
+// Upper bound of the true count behind an estimate est = scale * (sampled
+// count): five standard deviations of the sampling error plus slack.
+__device__ __forceinline__ double count_upper(double est, double scale) {
+  return est + 5.0 * sqrt(est * (scale - 1.0)) + 16.0;
+}
+
+// The smallest bucket whose estimated inclusive count, less five standard
+// deviations of its sampling error, reaches `need` (so the prefix of buckets
+// up to it holds at least `need` elements with high probability; the exact
+// pass checks it). Returns -1 when the prefix's upper bound exceeds `cap` or
+// no bucket qualifies.
+__device__ __noinline__ int plan_prefix_count(RSmem& sm, long long need, double scale, int cap) {
+  constexpr int PER = NB / RT;
+  const int base = (int)threadIdx.x * PER;
+  long long lc = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) lc += sm.cnt[base + i];
+  long long tc;
+  const long long pc = block_exscan<long long>(lc, sm.red_l, tc);
+  int mine = NB;
+  {
+    long long c = pc;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      c += sm.cnt[base + i];
+      const double est = scale * (double)c;
+      const double lower = scale > 1.0 ? est - 5.0 * sqrt(est * (scale - 1.0)) : est;
+      if (mine == NB && sm.cnt[base + i] > 0 && lower >= (double)need) mine = base + i;
+    }
+  }
+  const int b = block_min_i(mine, sm);
+  if (b >= NB - 1) return -1;  // never plan into the clamped far-tail bucket
+  if (threadIdx.x == b / PER) {
+    long long c = pc;
+    for (int i = base; i <= b; ++i) c += sm.cnt[i];
+    sm.bl[1] = c;
+  }
+  __syncthreads();
+  const long long incl = sm.bl[1];
+  __syncthreads();
+  if (count_upper(scale * (double)incl, scale) > (double)cap) return -1;
+  return b;
+}
+
+// The sample's estimate of the fraction of the row's mass in buckets below b
+// (every sampled element weighs its bucket's mid-point mass; the far-tail
+// bucket weighs 0).
+__device__ __noinline__ double estimated_mass_before(RSmem& sm, int b) {
+  const double wmid = sm.bd[3];
+  double v[2] = {0.0, 0.0};
+  for (int i = threadIdx.x; i < NB - 1; i += RT) {
+    const double w = (double)sm.cnt[i] * tab_at(sm.tab, i) * wmid;
+    v[0] += w;
+    v[1] += i < b ? w : 0.0;
+  }
+  block_sum_multi<2>(v, sm);
+  return v[0] > 0.0 ? v[1] / v[0] : 1.0;
+}
+
+// Highest bucket below b holding a sampled element (0 when none does).
+__device__ int sampled_before(RSmem& sm, int b) {
+  int mine = -1;
+  for (int i = threadIdx.x; i < b; i += RT)
+    if (sm.cnt[i] > 0) mine = i;
+  const int r = (int)block_ext_u<true>((unsigned long long)(mine + 1), sm) - 1;
+  return r < 0 ? 0 : r;
+}
+
+// Applies f to every key left in the per-warp gather slices of pass 2 (each
+// slice holds at most WCAP = RT keys, so a thread visits one key per slice).
+template <typename F>
+__device__ __forceinline__ void for_each_gathered(RSmem& sm, F&& f) {
+  static_assert(WCAP <= RT, "one key per thread per slice");
+  for (int w = 0; w < NWARP; ++w) {
+    const int cnt = min(sm.wcount[w], WCAP);
+    if ((int)threadIdx.x < cnt) f(sm.cand[w * WCAP + threadIdx.x]);
+  }
+}
+
+// Mass, count and smallest key of the gathered elements with key >= kt whose
+// bucket lies in [lo, hi] (the min-p range of the planned pass).
+__device__ __noinline__ void gathered_kept(RSmem& sm, float m, int lo, int hi, uint32_t kt,
+                                           double& mass, long long& cnt, unsigned long long& k_min,
+                                           double& qx) {
+  double ms = 0.0, c = 0.0, mx = 0.0;
+  unsigned long long kmn = ~0ull;
+  for_each_gathered(sm, [&](unsigned long long K) {
+    const float v = ckey_value(K);
+    const int b = bin0(v, m);
+    if (b < lo || b > hi || (uint32_t)(K >> 32) < kt) return;
+    const double q = qmass(sm, v, m);
+    ms += q;
+    mx += q * ((double)v - (double)m);
+    c += 1.0;
+    kmn = K < kmn ? K : kmn;
+  });
+  double s[3] = {ms, c, mx};
+  block_sum_multi<3>(s, sm);
+  mass = s[0];
+  cnt = (long long)s[1];
+  qx = s[2];
+  k_min = block_ext_u<false>(kmn, sm);
+}
+
+// On return, `sampled` tells whether sm.cnt holds the planning sample's counts
+// (the fast path then counts only the rest of the row).
+template <bool VEC>
+__device__ __noinline__ bool resolve_row_planned(RSmem& sm, const float* __restrict__ x, int V,
+                                                 float m, int k, float p, float mu, uint32_t kt,
+                                                 bool ent, bool& sampled, Cut& best) {
+  const bool k_on = k >= 1 && k < V, p_on = p < 1.0f, mu_on = mu > 0.0f;
+  sampled = false;
+  if (!k_on && !p_on && !mu_on) return false;  // identity rows: the fast path's single pass
+  const int ns = sample_hist<VEC>(sm, x, V, m);
+  sampled = true;
+  const double scale = (double)V / (double)ns;
+  Plan2 pl;
+  pl.need_last = 0;
+  pl.g_lo = 1;
+  pl.g_hi = 0;
+  pl.g2_lo = 1;
+  pl.g2_hi = 0;
+  pl.w_lo = -1;
+  pl.b_mu = -1;
+  pl.ent = ent ? 1 : 0;
+  Pass2 P;
+
+  if (k_on) {
+    // every bucket up to the one that holds the k-th element, by the sample
+    const int bk = plan_prefix_count(sm, (long long)k, scale, SCAP);
+    if (bk < 0) return false;
+    pl.g_lo = 0;
+    pl.g_hi = bk;
+    pass2<VEC>(sm, x, V, m, false, pl, P);
+    if (P.overflow) return false;
+    const int ng = pack_gathered(sm);
+    const int n = compact_gathered(sm, ng, m, 0, bk);
+    if (n < k || ng >= SCAP) return false;  // the prefix does not reach the k-th element
+    sort_and_scan(sm, n, m);
+    const int jk = k - 1;
+    Cut ck{sm.cand[jk], (long long)jk + 1, sm.cq[jk]};
+    best = ck;
+    if (p_on) {
+      const int jp = first_mass_hit(sm, 0, jk + 1, 0.0, 0.0, kMassGE, (double)p * ck.mass);
+      take_earlier(best, Cut{sm.cand[jp], (long long)jp + 1, sm.cq[jp]});
+    }
+    if (mu_on) {
+      int mine = 0;
+      for (int j = threadIdx.x; j < n; j += RT) mine += (uint32_t)(sm.cand[j] >> 32) >= kt ? 1 : 0;
+      const int nk = (int)block_sum_l(mine, sm);
+      if (nk >= 1 && nk < n) take_earlier(best, Cut{sm.cand[nk - 1], (long long)nk, sm.cq[nk - 1]});
+    }
+    if (ent) best.qx = sorted_prefix_qx(sm, (int)best.cnt, m);  // the support is a sorted prefix
+    __syncthreads();
+    return true;
+  }
+
+  // top-k off: min-p alone, or min-p with a top-p crossing that the sample
+  // puts clearly after the min-p prefix (the exact pass confirms it; rows
+  // where top-p decides take the fast path, which counts the rest of the row
+  // onto the sample). Everything in buckets below bm = bucket(threshold) is
+  // kept and everything above it dropped; the range gathered starts at the
+  // last sampled bucket before bm, which is non-empty, so it or bm holds the
+  // last kept element.
+  if (!mu_on) return false;
+  const int bm = bin0(key32_value(kt), m);
+  const int g2lo = sampled_before(sm, bm);
+  if (p_on && estimated_mass_before(sm, bm + 1) > (double)p - 0.05) return false;
+  const double est = scale * (double)count_range(sm, g2lo, bm + 1);
+  if (count_upper(est, scale) > 0.75 * CAP) return false;  // keep the warp slices far from full
+  MuPass mp;
+  mu_pass<VEC>(sm, x, V, m, g2lo, bm, ent, mp);
+  if (mp.overflow) return false;
+  double km, kx;
+  long long kc;
+  unsigned long long kmin;
+  gathered_kept(sm, m, g2lo, bm, kt, km, kc, kmin, kx);
+  if (kc == 0) return false;
+  const Cut cm{kmin, mp.cnt + kc, mp.mass + km, mp.qx + kx};
+  // With top-p on, the min-p prefix decides when its mass stays below p Z.
+  // Each element after the gathered range weighs at least tab[b] exp(-1/128)
+  // (less 1e-5 for the fp32 rounding of its bucket index), so
+  // Z >= (its mass) + that bound, which certifies it; otherwise the fast path.
+  const double rest_lower = mp.rest_upper * exp(-1.0 / 128.0) * (1.0 - 1e-5);
+  if (p_on && !(cm.mass < (double)p * (cm.mass + rest_lower))) return false;
+  best = cm;
+  return true;
+}
+
 template <bool VEC>
 __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   RSmem& sm = *reinterpret_cast<RSmem*>(smem_raw);
   const int V = a.V;
   init_exp_tab(sm.tab, threadIdx.x, RT);
-  if (threadIdx.x == 0) sm.bd[3] = exp(-1.0 / 256.0);  // mid-bucket weight factor
+  sm.ring_q[threadIdx.x] = 0;
+  if (threadIdx.x == 0) {
+    sm.bd[3] = exp(-1.0 / 256.0);  // mid-bucket weight factor
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(smem_u32(&sm.full_bar[s]), 1);
+      mbar_init(smem_u32(&sm.empty_bar[s]), NWARP);
+    }
+    sm.abort_flag = 0;
+    sm.err = &a.hdr->err;
+    fence_barrier_init();
+  }
   __syncthreads();
 
   // A row's metadata and the first two of its partial maxima per thread are
@@ -1436,6 +2112,7 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
       if (threadIdx.x == 0) {
         const float nan = __int_as_float(0x7fc00000);
         if (a.logprob) a.logprob[r] = nan;
+        if (a.entropy) a.entropy[r] = nan;
         if (a.row_max) a.row_max[r] = nan;
         if (a.lse_support) a.lse_support[r] = nan;
         if (a.cut_logit) a.cut_logit[r] = nan;
@@ -1479,14 +2156,31 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
 
     Cut best;
     bool hist_valid = false;
-    bool ok = resolve_row_fast<VEC>(sm, x, V, m, k, p, mu, kt, best);
-    if (!ok) ok = resolve_row_exact<VEC>(sm, x, V, m, k, p, mu, kt, hist_valid, best);
+    // planned pass first; the fast path and the exact search decide the rows
+    // whose plan does not hold (identity rows go straight to the fast path's
+    // single pass)
+    int path = (k_on || p_on || mu_on) ? kPathPlanned : kPathIdentity;
+    bool sampled = false;
+    const bool ent = a.entropy != nullptr;
+    bool ok = resolve_row_planned<VEC>(sm, x, V, m, k, p, mu, kt, ent, sampled, best);
+    if (!ok) {
+      if (path == kPathPlanned) path = kPathFast;
+      ok = resolve_row_fast<VEC>(sm, x, V, m, k, p, mu, kt, sampled, ent, best);
+    }
+    if (!ok) {
+      path = kPathExact;
+      ok = resolve_row_exact<VEC>(sm, x, V, m, k, p, mu, kt, hist_valid, best);
+    }
+    if (threadIdx.x == 0) atomicAdd(&a.hdr->path_rows[path], 1ull);
+    __syncthreads();
+    if (sm.abort_flag) break;  // a bounded wait gave up: STS_ERR_TIMEOUT is recorded
 
     if (!ok) {  // a bound of the exact search was exceeded: the row fails like an invalid one
       if (threadIdx.x == 0) {
         atomicCAS(&a.hdr->err, 0, (int)STS_ERR_OVERFLOW);
         const float nan = __int_as_float(0x7fc00000);
         if (a.logprob) a.logprob[r] = nan;
+        if (a.entropy) a.entropy[r] = nan;
         if (a.row_max) a.row_max[r] = nan;
         if (a.lse_support) a.lse_support[r] = nan;
         if (a.cut_logit) a.cut_logit[r] = nan;
@@ -1502,6 +2196,12 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
     }
 
     const double lse = md + log(best.mass);
+    if (ent) {
+      // entropy of the renormalised support: ln Z_S - sum_S q (s - m) / Z_S,
+      // q = exp(s - m); the sum comes from the deciding path, else one pass
+      const double qx = isnan(best.qx) ? support_qx_pass<VEC>(sm, x, V, m, best.K) : best.qx;
+      if (threadIdx.x == 0) a.entropy[r] = (float)fmax(log(best.mass) - qx / best.mass, 0.0);
+    }
     if (a.mode == kModeSample) {
       Cut cs;
       const double tgt = a.u[r] * best.mass;

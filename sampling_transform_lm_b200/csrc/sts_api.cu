@@ -12,6 +12,7 @@
 // "Self-review pass" single-pass vocabulary-chunked backward with write-once
 // weight-gradient slices.)
 #include <algorithm>
+#include <cstddef>
 #include <atomic>
 #include <cstring>
 #include <mutex>
@@ -247,7 +248,9 @@ sts_status reset_header(void* ws, cudaStream_t st) {
   WsHeader* h = static_cast<WsHeader*>(ws);
   if (cudaMemsetAsync(&h->bad_row_code, 0xFF, sizeof(h->bad_row_code), st) != cudaSuccess)
     return STS_ERR_CUDA;
-  if (cudaMemsetAsync(&h->err, 0, sizeof(h->err), st) != cudaSuccess) return STS_ERR_CUDA;
+  // err, its padding and the path counters are contiguous
+  static_assert(offsetof(WsHeader, path_rows) == offsetof(WsHeader, err) + 8, "header layout");
+  if (cudaMemsetAsync(&h->err, 0, 8 + sizeof(h->path_rows), st) != cudaSuccess) return STS_ERR_CUDA;
   return STS_OK;
 }
 
@@ -264,8 +267,8 @@ sts_status reset_header(void* ws, cudaStream_t st) {
 
 // Forward-style pass shared by sts_forward and sts_sample.
 sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, const sts_rows* rows,
-                        float* logprob, const sts_saved* saved, const double* u, int64_t* sampled,
-                        void* ws, size_t ws_bytes, cudaStream_t st) {
+                        float* logprob, float* entropy, const sts_saved* saved, const double* u,
+                        int64_t* sampled, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (!shape_ok(shape)) return STS_ERR_SHAPE;
   if (!H || !W) return STS_ERR_NULL;
   const bool fwd = (sampled == nullptr);
@@ -334,6 +337,7 @@ sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, co
     a.flags_out = flags + t0;
     if (fwd) {
       a.logprob = logprob + t0;
+      a.entropy = entropy ? entropy + t0 : nullptr;
       a.row_max = saved->row_max + t0;
       a.lse_support = saved->lse_support + t0;
       a.cut_logit = saved->cut_logit + t0;
@@ -396,9 +400,9 @@ size_t sts_workspace_bytes(const sts_shape* shape, int pass) {
 }
 
 sts_status sts_forward(const sts_shape* shape, const void* H, const void* W, const sts_rows* rows,
-                       float* logprob, const sts_saved* saved, void* ws, size_t ws_bytes,
-                       sts_stream_t stream) {
-  return forward_impl(shape, H, W, rows, logprob, saved, nullptr, nullptr, ws, ws_bytes,
+                       float* logprob, float* entropy, const sts_saved* saved, void* ws,
+                       size_t ws_bytes, sts_stream_t stream) {
+  return forward_impl(shape, H, W, rows, logprob, entropy, saved, nullptr, nullptr, ws, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -406,14 +410,17 @@ sts_status sts_sample(const sts_shape* shape, const void* H, const void* W, cons
                       const double* u, int64_t* sampled, void* ws, size_t ws_bytes,
                       sts_stream_t stream) {
   if (!sampled) return STS_ERR_NULL;
-  return forward_impl(shape, H, W, rows, nullptr, nullptr, u, sampled, ws, ws_bytes,
+  return forward_impl(shape, H, W, rows, nullptr, nullptr, nullptr, u, sampled, ws, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
-sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, const sts_rows* rows,
-                        const sts_saved* saved, const float* grad, float* dH, float* dW,
-                        int accumulate_dW, void* ws, size_t ws_bytes, sts_stream_t stream) {
+sts_status sts_backward_sliced(const sts_shape* shape, const void* H, const void* W,
+                               const sts_rows* rows, const sts_saved* saved, const float* grad,
+                               float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
+                               sts_stream_t stream, sts_slice_fn on_dw_slice, void* user,
+                               int comm_sms) {
   if (!shape_ok(shape)) return STS_ERR_SHAPE;
+  if (comm_sms < 0) return STS_ERR_SHAPE;
   if (!H || !W || !grad || !dH || !dW) return STS_ERR_NULL;
   STS_TRY(check_rows(shape, rows, true));
   if (!saved || !saved->lse_support || !saved->cut_logit || !saved->cut_id || !saved->flags)
@@ -423,6 +430,8 @@ sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, co
   STS_TRY(check_ws(ws, ws_bytes, L.total));
   DeviceInfo dev;
   STS_TRY(device_info(dev));
+  if (comm_sms >= dev.sms) return STS_ERR_SHAPE;
+  dev.sms -= comm_sms;  // persistent GEMMs leave these SMs to the caller's exchange kernels
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
   const int64_t T = shape->T, V = shape->V, d = shape->d, Vc = vocab_chunk(shape);
@@ -474,6 +483,9 @@ sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, co
       return accumulate_dW ? run_gemm<true, true, kEpiReduceF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st)
                            : run_gemm<true, true, kEpiStoreF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st);
     }));
+    // the slice is final once this GEMM completes on `st`: hand it out before
+    // enqueuing the work that follows, so its exchange overlaps that work
+    if (on_dw_slice) on_dw_slice(user, v0, w, dW + (size_t)v0 * (size_t)d, stream);
 
     // 3. dH (+)= dZ . W[v0:v0+w] (W read MN-major)
     GemmParams r{};
@@ -490,9 +502,17 @@ sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, co
   return STS_OK;
 }
 
+sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, const sts_rows* rows,
+                        const sts_saved* saved, const float* grad, float* dH, float* dW,
+                        int accumulate_dW, void* ws, size_t ws_bytes, sts_stream_t stream) {
+  return sts_backward_sliced(shape, H, W, rows, saved, grad, dH, dW, accumulate_dW, ws, ws_bytes,
+                             stream, nullptr, nullptr, 0);
+}
+
 sts_status sts_filter_logits(const sts_shape* shape, const float* S, const sts_rows* rows,
                              int32_t* support_size, float* cut_logit, int32_t* cut_id,
-                             uint8_t* mask, void* ws, size_t ws_bytes, sts_stream_t stream) {
+                             uint8_t* mask, float* entropy, void* ws, size_t ws_bytes,
+                             sts_stream_t stream) {
   if (!shape_ok(shape)) return STS_ERR_SHAPE;
   if (!S || !support_size || !cut_logit || !cut_id) return STS_ERR_NULL;
   if (!rows) return STS_ERR_NULL;
@@ -525,6 +545,7 @@ sts_status sts_filter_logits(const sts_shape* shape, const float* S, const sts_r
   a.cut_logit = cut_logit;
   a.cut_id = cut_id;
   a.mask = mask;
+  a.entropy = entropy;
   a.hdr = hdr;
   STS_CUDA(timed_launch(STS_KERNEL_RESOLVE, st, [&] { return launch_resolve(a, dev.sms, st); }));
   return STS_OK;
@@ -558,6 +579,15 @@ sts_status sts_scaled_logits(const sts_shape* shape, const void* H, const void* 
   STS_CUDA(timed_launch(STS_KERNEL_LOGITS_GEMM, st, [&] {
     return run_gemm<false, false, kEpiLogits>(ma, mb, mc, p, dev.sms, st);
   }));
+  return STS_OK;
+}
+
+sts_status sts_path_counts(const void* ws, sts_stream_t stream, int64_t* counts) {
+  if (!ws || !counts) return STS_ERR_NULL;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return STS_ERR_CUDA;
+  WsHeader h;
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return STS_ERR_CUDA;
+  for (int i = 0; i < 4; ++i) counts[i] = (int64_t)h.path_rows[i];
   return STS_OK;
 }
 

@@ -13,11 +13,14 @@ namespace sts {
 // Status header at the start of every workspace (256 bytes).
 //   bad_row_code: min over failing rows of (row << 32 | status); all-ones = none
 //   err:          first non-row error (timeout, overflow), 0 = none
+//   path_rows:    rows the resolver decided by each path (diagnostic counters)
+enum ResolvePath : int { kPathPlanned = 0, kPathFast = 1, kPathExact = 2, kPathIdentity = 3 };
 struct WsHeader {
   unsigned long long bad_row_code;
   int err;
   int pad0;
-  unsigned long long reserved[30];
+  unsigned long long path_rows[4];
+  unsigned long long reserved[26];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
@@ -42,6 +45,7 @@ struct ResolveArgs {
   const int32_t* row_flags;  // validation result (STS_ROW_INVALID bit)
   // outputs (chunk-offset); any may be null when the mode does not use it
   float* logprob;
+  float* entropy;          // forward: entropy of the filtered distribution, or null
   float* row_max;
   float* lse_support;
   float* cut_logit;

@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol(lib):
     for name in names:
         assert hasattr(lib, name), name
     assert set(names) == set(sts.EXPORTED_SYMBOLS)
-    assert lib.sts_abi_version() == 1
+    assert lib.sts_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -70,7 +70,7 @@ def test_bad_shapes_rejected(lib, bad):
     assert lib.sts_workspace_bytes(ctypes.byref(sh), 0) == 0
     rows = _Rows(kw["T"], 16, 16, 16, 16, 16)
     saved = _Saved(16, 16, 16, 16, 16, 16)
-    st = lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(rows), 16, ctypes.byref(saved),
+    st = lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(rows), 16, None, ctypes.byref(saved),
                          4096, 1 << 40, None)
     assert st == 2  # STS_ERR_SHAPE
 
@@ -81,24 +81,32 @@ def test_null_and_length_and_workspace_errors(lib):
     good_rows = _Rows(256, 16, 16, 16, 16, 16)
     big = 1 << 40
     # null operands
-    assert lib.sts_forward(ctypes.byref(sh), None, 4096, ctypes.byref(good_rows), 16,
+    assert lib.sts_forward(ctypes.byref(sh), None, 4096, ctypes.byref(good_rows), 16, None,
                            ctypes.byref(saved), 4096, big, None) == 1
     # metadata length differs from T: rejected, not truncated
     for n in (255, 257, 512):
         rows = _Rows(n, 16, 16, 16, 16, 16)
-        assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(rows), 16,
+        assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(rows), 16, None,
                                ctypes.byref(saved), 4096, big, None) == 2
     # missing per-row array
     rows = _Rows(256, 16, None, 16, 16, 16)
-    assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(rows), 16,
+    assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(rows), 16, None,
                            ctypes.byref(saved), 4096, big, None) == 1
     # workspace: null, misaligned, too small
-    assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(good_rows), 16,
+    assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(good_rows), 16, None,
                            ctypes.byref(saved), None, big, None) == 9
-    assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(good_rows), 16,
+    assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(good_rows), 16, None,
                            ctypes.byref(saved), 4096 + 16, big, None) == 9
-    assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(good_rows), 16,
+    assert lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(good_rows), 16, None,
                            ctypes.byref(saved), 4096, 1024, None) == 9
+    # sliced backward: a negative SM reservation is a shape error
+    SLICE = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                             ctypes.c_void_p, ctypes.c_void_p)
+    lib.sts_backward_sliced.argtypes = [ctypes.c_void_p] * 12 + [SLICE, ctypes.c_void_p,
+                                                                 ctypes.c_int]
+    assert lib.sts_backward_sliced(ctypes.byref(sh), 4096, 4096, ctypes.byref(good_rows),
+                                   ctypes.byref(saved), 4096, 4096, 4096, 0, 4096, big, None,
+                                   SLICE(0), None, -1) == 2
     # backward: null gradient
     assert lib.sts_backward(ctypes.byref(sh), 4096, 4096, ctypes.byref(good_rows),
                             ctypes.byref(saved), None, 4096, 4096, 0, 4096, big, None) == 1
@@ -116,7 +124,7 @@ def test_valid_call_without_gpu_reports_cuda_error(lib):
     sh = _shape()
     saved = _Saved(16, 16, 16, 16, 16, 16)
     rows = _Rows(256, 16, 16, 16, 16, 16)
-    st = lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(rows), 16, ctypes.byref(saved),
+    st = lib.sts_forward(ctypes.byref(sh), 4096, 4096, ctypes.byref(rows), 16, None, ctypes.byref(saved),
                          4096, 1 << 40, None)
     assert st in (12, 13)  # no device: CUDA error, never a CPU fallback
 

@@ -15,7 +15,10 @@ Checks, each able to fail on any sampled row:
      same rows (same fp32 values, every decision in float64 on both sides);
      a difference is only allowed where that row's top-p crossing is within
      1e-12 of a boundary (float64 summation order);
-  4. dH on the sampled rows and dW on ~1000 sampled vocabulary rows (the
+  4. the entropy of each filtered distribution (the forward's optional
+     output) against the oracle's: within 1e-3 on the float64 logits and the
+     GPU's support, and to fp32 rounding on the GPU's own fp32 logits;
+  5. dH on the sampled rows and dW on ~1000 sampled vocabulary rows (the
      upstream gradient is 1 on the sampled rows whose support equals the
      oracle's, 0 elsewhere, so dW stays comparable): relative Frobenius
      error < 1e-2.
@@ -73,7 +76,7 @@ def test_full_size_workload(cuda_lib, pool, index):
     y_t = dev(target, np.int64)
     tau, k, p, mu = (dev(data["temperature"], np.float32), dev(data["top_k"], np.int32),
                      dev(data["top_p"], np.float32), dev(data["min_p"], np.float32))
-    lp, saved, _ = sts.sts_forward(Hd, Wd, y_t, tau, k, p, mu, check=True)
+    lp, saved, _ = sts.sts_forward(Hd, Wd, y_t, tau, k, p, mu, check=True, entropy=True)
     lp_sel = lp.cpu().numpy()[sel]
     sv = {n: v.cpu().numpy()[sel] for n, v in saved.items()}
 
@@ -96,8 +99,16 @@ def test_full_size_workload(cuda_lib, pool, index):
           f"{int((~cut_diff).sum())} of {n} rows")
     assert bad == 0
     assert not (cut_diff & ~(own_gap_p < 1e-12)).any(), np.flatnonzero(cut_diff)
+    # entropy of the filtered distribution: against the oracle's on the GPU's
+    # support (float64 logits) and on the GPU's own fp32 logits
+    ent_ref = np.concatenate(pool.map_rows("entropy", s_sel, rows_sel,
+                                           per_row_extra=(sv["support_size"],)))
+    assert np.abs(sv["entropy"] - ent_ref).max() < 1e-3
+    ent_own = np.concatenate(pool.map_rows("entropy", S_gpu, rows_sel))
+    same_cut = ~cut_diff
+    np.testing.assert_allclose(sv["entropy"][same_cut], ent_own[same_cut], rtol=2e-6, atol=1e-6)
 
-    # 4: gradients on the rows whose support equals the oracle's; zero elsewhere
+    # 5: gradients on the rows whose support equals the oracle's; zero elsewhere
     same = grad_rows(sv["flags"], ref["in_support"]) & (dsize == 0)
     g = np.zeros(T, np.float32)
     g[sel[same]] = 1.0

@@ -111,6 +111,30 @@ def _filter_case():
     add(rng.standard_normal(V).astype(np.float32), 0, float(np.nextafter(np.float32(1), np.float32(0))), 0.0)
     add(rng.standard_normal(V).astype(np.float32), V, 1.0, 0.0)
     add(rng.standard_normal(V).astype(np.float32), -3, 1.0, 0.01)
+    # the planning sample reads float4 sweeps 0, 8, 16, ... of 512 float4s:
+    # elements [0, 2048) and [16384, 18432) here. Rows whose sample is
+    # unrepresentative must still resolve exactly (the plan is only checked).
+    skew = rng.standard_normal(V).astype(np.float32)
+    skew[:2048] -= 6.0
+    skew[16384:18432] -= 6.0
+    add(skew, 0, 0.9, 0.0)
+    add(skew, 30, 0.9, 0.05)
+    add(skew, 0, 1.0, 0.2)
+    hot = rng.standard_normal(V).astype(np.float32) - 4.0
+    hot[:2048] += 6.0  # the sample sees only the top of the row
+    add(hot, 0, 0.7, 0.0)
+    add(hot, 100, 1.0, 0.0)
+    add(rng.standard_normal(V).astype(np.float32), 0, 1.0, 1e-30)  # threshold in the far tail
+    peaked = (rng.standard_normal(V) * 0.01 - 30.0).astype(np.float32)
+    peaked[123] = 0.0  # min-p keeps the max alone; no sampled bucket before it
+    add(peaked, 0, 1.0, 0.5)
+    add(peaked, 0, 0.5, 0.5)
+    # large top-k (more than the 4096-entry sort up to the k-th element's
+    # bucket): the k-th element inside its own bucket, then top-p on the
+    # top-k mass and min-p before, at or after that bucket
+    for kk in (6000, 9000, 15000):
+        for pp, mm in ((1.0, 0.0), (0.9, 0.0), (1.0, 0.02), (0.95, 0.3)):
+            add(rng.standard_normal(V).astype(np.float32), kk, pp, mm)
     S = np.stack(rows)
     T = S.shape[0]
     md = {
@@ -123,13 +147,22 @@ def _filter_case():
     return S, md
 
 
+ENT_RTOL, ENT_ATOL = 2e-6, 1e-6  # fp32 output of a float64 sum on the same fp32 logits
+
+
+def _check_entropy(got, S, md):
+    want = oracle.entropy(S, md)
+    np.testing.assert_allclose(got.cpu().numpy(), want, rtol=ENT_RTOL, atol=ENT_ATOL)
+
+
 def test_filter_bit_exact_against_oracle(cuda_lib):
     sts = cuda_lib
     S, md = _filter_case()
     T, V = S.shape
     out = sts.sts_filter_logits(torch.from_numpy(S).cuda(), torch.from_numpy(md["top_k"]).cuda(),
                                 torch.from_numpy(md["top_p"]).cuda(),
-                                torch.from_numpy(md["min_p"]).cuda(), want_mask=True, check=True)
+                                torch.from_numpy(md["min_p"]).cuda(), want_mask=True,
+                                want_entropy=True, check=True)
     ref = oracle.filter_rows(S, md, want_mask=True)
     size = out["size"].cpu().numpy()
     cid = out["cut_id"].cpu().numpy()
@@ -139,6 +172,35 @@ def test_filter_bit_exact_against_oracle(cuda_lib):
     assert not bad, [(t, size[t], ref["size"][t], cid[t], ref["cut_id"][t]) for t in bad]
     assert np.array_equal(cval, S[np.arange(T), ref["cut_id"]])
     assert np.array_equal(mask, ref["mask"])
+    # the entropy of each filtered distribution, every resolver path included
+    _check_entropy(out["entropy"], S, md)
+
+
+def test_filter_odd_vocab_scalar_path(cuda_lib):
+    """A row stride that is not a multiple of four floats takes the scalar
+    load path of every pass (planning sample included): bit-exact too."""
+    sts = cuda_lib
+    rng = np.random.Generator(np.random.PCG64(81))
+    T, V = 40, 7001
+    S = (rng.standard_normal((T, V), dtype=np.float32)
+         / rng.uniform(0.4, 1.6, T).astype(np.float32)[:, None])
+    S[5:10, ::7] = S[5:10, :1]  # exact ties
+    md = {
+        "top_k": rng.choice(np.array([0, 1, 20, 700, 7001], np.int32), T).astype(np.int32),
+        "top_p": rng.choice(np.array([1.0, 0.95, 0.6, 0.2], np.float32), T).astype(np.float32),
+        "min_p": rng.choice(np.array([0.0, 0.02, 0.3], np.float32), T).astype(np.float32),
+        "temperature": np.ones(T, np.float32),
+        "target": np.zeros(T, np.int64),
+    }
+    out = sts.sts_filter_logits(torch.from_numpy(S).cuda(), torch.from_numpy(md["top_k"]).cuda(),
+                                torch.from_numpy(md["top_p"]).cuda(),
+                                torch.from_numpy(md["min_p"]).cuda(), want_mask=True,
+                                want_entropy=True, check=True)
+    ref = oracle.filter_rows(S, md, want_mask=True)
+    assert np.array_equal(out["size"].cpu().numpy(), ref["size"])
+    assert np.array_equal(out["cut_id"].cpu().numpy(), ref["cut_id"])
+    assert np.array_equal(out["mask"].cpu().numpy().astype(bool), ref["mask"])
+    _check_entropy(out["entropy"], S, md)
 
 
 def test_filter_flat_rows_full_vocab(cuda_lib):
@@ -157,9 +219,15 @@ def test_filter_flat_rows_full_vocab(cuda_lib):
         "target": np.zeros(T, np.int64),
     }
     md["top_p"][::5] = 1.0
+    ws = torch.empty(sts.sts_workspace_bytes(T, 8, V, 2), dtype=torch.uint8, device="cuda")
     out = sts.sts_filter_logits(torch.from_numpy(S).cuda(), torch.from_numpy(md["top_k"]).cuda(),
                                 torch.from_numpy(md["top_p"]).cuda(),
-                                torch.from_numpy(md["min_p"]).cuda(), check=True)
+                                torch.from_numpy(md["min_p"]).cuda(), ws=ws, check=True)
+    paths = sts.sts_path_counts(ws)
+    print("resolver paths:", paths)
+    assert sum(paths.values()) == T
+    # top-k rows are decided by the sampled plan and one gathering pass
+    assert paths["planned"] >= int((md["top_k"] > 0).sum()), paths
     ref = oracle.filter_rows(S, md)
     gaps = oracle.row_gaps(S, md).min(axis=1)
     size = out["size"].cpu().numpy()
@@ -167,6 +235,41 @@ def test_filter_flat_rows_full_vocab(cuda_lib):
     mism = (size != ref["size"]) | (cid != ref["cut_id"])
     # a mismatch is only acceptable where float64 summation order could decide it
     assert not (mism & (gaps > 1e-12)).any(), np.flatnonzero(mism)
+
+
+def test_large_top_k_takes_the_direct_path(cuda_lib):
+    """Headline-shaped rows with top-k between 4096 and V: decided by the
+    count pass and one exact pass (the k-th element located in its bucket),
+    not by the exact search; bit-exact against the oracle."""
+    sts = cuda_lib
+    rng = np.random.Generator(np.random.PCG64(82))
+    T, V = 12, 152064
+    S = (rng.standard_normal((T, V), dtype=np.float32)
+         / rng.uniform(0.6, 1.4, T).astype(np.float32)[:, None])
+    md = {
+        "top_k": np.array([5000, 20000, 70000, 150000] * 3, np.int32),
+        "top_p": np.array([1.0] * 8 + [0.9] * 4, np.float32),
+        "min_p": np.array([0.0] * 4 + [0.05] * 4 + [0.0] * 4, np.float32),
+        "temperature": np.ones(T, np.float32),
+        "target": np.zeros(T, np.int64),
+    }
+    ws = torch.empty(sts.sts_workspace_bytes(T, 8, V, 2), dtype=torch.uint8, device="cuda")
+    out = sts.sts_filter_logits(torch.from_numpy(S).cuda(), torch.from_numpy(md["top_k"]).cuda(),
+                                torch.from_numpy(md["top_p"]).cuda(),
+                                torch.from_numpy(md["min_p"]).cuda(), ws=ws, want_entropy=True,
+                                check=True)
+    paths = sts.sts_path_counts(ws)
+    print("resolver paths:", paths)
+    assert paths["exact"] == 0, paths
+    ref = oracle.filter_rows(S, md)
+    gaps = oracle.row_gaps(S, md).min(axis=1)
+    size = out["size"].cpu().numpy()
+    cid = out["cut_id"].cpu().numpy()
+    mism = (size != ref["size"]) | (cid != ref["cut_id"])
+    assert not (mism & (gaps > 1e-12)).any(), np.flatnonzero(mism)
+    ok = ~mism
+    np.testing.assert_allclose(out["entropy"].cpu().numpy()[ok], oracle.entropy(S, md)[ok],
+                               rtol=ENT_RTOL, atol=ENT_ATOL)
 
 
 def _estimate_defeating_rows():
@@ -216,9 +319,16 @@ def _estimate_defeating_rows():
 def test_filter_when_the_planning_estimate_is_wrong(cuda_lib):
     sts = cuda_lib
     S, md = _estimate_defeating_rows()
+    T, V = S.shape
+    ws = torch.empty(sts.sts_workspace_bytes(T, 8, V, 2), dtype=torch.uint8, device="cuda")
     out = sts.sts_filter_logits(torch.from_numpy(S).cuda(), torch.from_numpy(md["top_k"]).cuda(),
                                 torch.from_numpy(md["top_p"]).cuda(),
-                                torch.from_numpy(md["min_p"]).cuda(), check=True)
+                                torch.from_numpy(md["min_p"]).cuda(), ws=ws, want_entropy=True,
+                                check=True)
+    paths = sts.sts_path_counts(ws)
+    print("resolver paths:", paths)
+    assert paths["fast"] + paths["exact"] > 0  # the fallbacks are exercised
+    _check_entropy(out["entropy"], S, md)
     ref = oracle.filter_rows(S, md)
     assert oracle.row_gaps(S, md).min() > 1e-6  # no near-tie decides these rows
     T = S.shape[0]

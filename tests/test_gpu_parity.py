@@ -10,16 +10,19 @@ import torch
 
 import oracle
 import workloads
+from sampling_transform_lm_b200.dp import SliceAllReduce
 from helpers import (GRAD_RTOL, bf16_tensor, compare_logprob, f32_values, grad_rows,
                      near_gap_rows, rel_fro, row_tensors, small_case)
 
 pytestmark = pytest.mark.gpu
 
+ENT_ATOL = 1e-3  # entropy from fp32-accumulated logits against float64 ones
+
 
 def _run(sts, H, W, rows, grad=None, row_chunk=0, vocab_chunk=0):
     Hd, Wd = bf16_tensor(H), bf16_tensor(W)
     y, tau, k, p, mu = row_tensors(rows)
-    lp, saved, ws = sts.sts_forward(Hd, Wd, y, tau, k, p, mu, row_chunk=row_chunk)
+    lp, saved, ws = sts.sts_forward(Hd, Wd, y, tau, k, p, mu, row_chunk=row_chunk, entropy=True)
     status, bad = sts.sts_get_status(ws)
     out = {"logprob": lp.cpu().numpy(), "saved": {k_: v.cpu().numpy() for k_, v in saved.items()},
            "status": status, "bad_row": bad}
@@ -49,6 +52,9 @@ def _check_forward(sts_out, s, rows, ref):
           f"{int(flagged.sum())} near-gap, {ndiff} of them with another valid support size")
     assert sts_out["status"] == 0
     assert bad == 0, (bad, ndiff, max_err)
+    # entropy of the filtered distribution on the GPU's support
+    ent = oracle.entropy(s, rows, sizes=size)
+    np.testing.assert_allclose(sts_out["saved"]["entropy"], ent, rtol=0, atol=ENT_ATOL)
     # gradients are comparable where the support is the oracle's
     return grad_rows(sts_out["saved"]["flags"], ref["in_support"]) & (size == ref["size"])
 
@@ -304,3 +310,40 @@ def test_policy_gradient_through_the_backward(cuda_lib):
     dH, dW = oracle.backward(Hf, Wf, rows, np.where(same, g_ref, 0.0), s=s)
     assert rel_fro(out["dH"], dH) < GRAD_RTOL
     assert rel_fro(out["dW"], dW) < GRAD_RTOL
+
+
+def test_sliced_backward_allreduce_single_rank(cuda_lib):
+    """sts_backward_sliced through SliceAllReduce on a one-rank NCCL group:
+    the hook sees every vocabulary slice once in increasing order, the result
+    equals the plain backward bit for bit (a one-rank sum is the identity),
+    and leaving SMs to the exchange does not change it either."""
+    import datetime
+    import socket
+
+    import torch.distributed as dist
+
+    sts = cuda_lib
+    H, W, meta, u = small_case(21, 300, 136, 2500)
+    Hf, Wf, s, rows = _oracle_case(H, W, meta, u)
+    Hd, Wd = bf16_tensor(H), bf16_tensor(W)
+    y, tau, k, p, mu = row_tensors(rows)
+    lp, saved, _ = sts.sts_forward(Hd, Wd, y, tau, k, p, mu, check=True)
+    g = torch.ones(300, dtype=torch.float32, device="cuda")
+    dH0, dW0 = sts.sts_backward(Hd, Wd, y, tau, k, p, mu, saved, g, vocab_chunk=512, check=True)
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        red = SliceAllReduce()
+        dH1, dW1 = sts.sts_backward(Hd, Wd, y, tau, k, p, mu, saved, g, vocab_chunk=512,
+                                    on_dw_slice=red, comm_sms=16, check=True)
+        order = red.finish()
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    assert order == [(v0, min(512, 2500 - v0)) for v0 in range(0, 2500, 512)]
+    assert torch.equal(dW1, dW0) and torch.equal(dH1, dH0)
