@@ -128,7 +128,7 @@ struct RSmem {
   long long bl[4];
   int bi[4];
   int ncand;
-  int wcount[NWARP];  // fast path: fill level of each warp's gather slice
+  int tcount[RT];     // gathered keys of each thread (slot j of thread t: cand[j RT + t])
 };
 
 // ---------------------------------------------------------------- keys
@@ -1036,7 +1036,7 @@ struct Plan2 {
   int ent;                  // also sum exp(s - m) (s - m) per region (entropy)
 };
 
-constexpr int WCAP = CAP / NWARP;  // private gather slots per warp
+constexpr int TCAP = CAP / RT;  // private gather slots per thread, interleaved across threads
 
 // One pass over the row: exact float64 masses accumulated in registers, and
 // the elements of up to two bucket ranges gathered into per-warp slices of
@@ -1053,15 +1053,14 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
   const bool need_last = pl.need_last != 0;
   const int g_lo = pl.g_lo, g_hi = pl.g_hi, g2_lo = pl.g2_lo, g2_hi = pl.g2_hi;
   const int w_lo = pl.w_lo, b_mu = pl.b_mu;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // gather ranges as (start, span) for one unsigned compare each; an empty
   // range (lo > hi) gets a start no bucket reaches
   const unsigned g1s = g_lo <= g_hi ? (unsigned)g_lo : 0x80000000u;
   const unsigned g1n = g_lo <= g_hi ? (unsigned)(g_hi - g_lo) : 0u;
   const unsigned g2s = g2_lo <= g2_hi ? (unsigned)g2_lo : 0x80000000u;
   const unsigned g2n = g2_lo <= g2_hi ? (unsigned)(g2_hi - g2_lo) : 0u;
-  unsigned long long* wbuf = sm.cand + warp * WCAP;
-  int wfill = 0;  // warp-uniform
+  unsigned long long* tbuf = sm.cand + threadIdx.x;  // this thread's slots, stride RT
+  int tfill = 0;
   double z[2] = {0.0, 0.0}, ap[2] = {0.0, 0.0}, amu[2] = {0.0, 0.0};
   double zx = 0.0, apx = 0.0, amux = 0.0;  // the same sums of q (s - m) (entropy)
   const bool ent = pl.ent != 0;
@@ -1152,23 +1151,14 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
       const bool g = ok(e) && (b - g1s <= g1n || b - g2s <= g2n);
       gm |= g ? 1u << e : 0u;
     }
-    // One slot range per thread from a warp scan of its hit count (hits are
-    // rare: a vote skips batches without any), then the hits stored in order.
+    // hits are rare: a vote skips batches without any; each thread appends to
+    // its own slots (no coordination between lanes)
     if (__any_sync(0xffffffffu, gm != 0u)) {
-      const int c = __popc(gm);
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int slot = wfill + incl - c;
-      wfill += __shfl_sync(0xffffffffu, incl, 31);
 #pragma unroll
       for (int e = 0; e < E; ++e)
         if ((gm >> e) & 1u) {
-          if (slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
-          ++slot;
+          if (tfill < TCAP) tbuf[tfill * RT] = ckey(sv[e], idx(e));
+          ++tfill;
         }
     }
   };
@@ -1195,7 +1185,7 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
     const float sv[E] = {t, t, t, t, t, t, t, t};
     batch(std::false_type{}, sv, i, in ? 1 : 0, i, 0);
   }
-  if (lane == 0) sm.wcount[warp] = wfill;
+  sm.tcount[threadIdx.x] = tfill;
   {
     double sums[8] = {z[0] + z[1], ap[0] + ap[1], amu[0] + amu[1], (double)cp, (double)cmu,
                       zx, apx, amux};
@@ -1210,10 +1200,7 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
     P.a_mux = sums[7];
   }
   P.k_last = need_last ? block_ext_u<false>(kl, sm) : ~0ull;
-  int ovf = 0;
-  for (int w = 0; w < NWARP; ++w) ovf |= sm.wcount[w] > WCAP ? 1 : 0;
-  P.overflow = ovf != 0;
-  __syncthreads();
+  P.overflow = __syncthreads_or(tfill > TCAP) != 0;
 }
 
 template <bool VEC>
@@ -1234,117 +1221,97 @@ __device__ void pass2(RSmem& sm, const float* __restrict__ x, int V, float m, bo
 
 // ---------------------------------------------------------------- min-p pass
 // One pass for a row whose min-p prefix decides the support. Elements in
-// buckets below g_lo are all kept: their values are compacted per warp into a
-// staging area and weighed in float64 in full batches (so the float64 work
+// buckets below g_lo are all kept: each thread stages their values in its
+// own slots and weighs them in float64 eight at a time (so the float64 work
 // follows the kept elements, not the row). Elements in buckets [g_lo, g_hi]
 // are gathered (their keys decide which are kept). Elements after g_hi are
-// dropped: they only add tab[b] per element to a lower bound of their mass,
-// exact since each weighs at least tab[b] exp(-1/128) and at most tab[b].
+// dropped: they only add to a lower bound of their mass, each at least
+// tab[b] exp(-1/128) = 2^(-(b + 1) log2(e) / 128), summed in fp32.
 struct MuPass {
   double mass, qx;     // kept elements before g_lo: mass and sum of q (s - m)
   long long cnt;       // their number
-  double rest_upper;   // sum of tab[b] over the elements after g_hi
-  bool overflow;       // a gather slice or the staging area overflowed
+  double rest_lower;   // lower bound of the mass of the elements after g_hi
+  bool overflow;       // the gather slots overflowed
 };
 
-constexpr int MU_STAGE = 512;  // staged values per warp (the storage of sm.mass)
-static_assert(NWARP * MU_STAGE * 4 <= NB * 8, "the staging area fits the bucket-mass storage");
+constexpr int MU_SLOTS = NB * 8 / 4 / RT;  // staged fp32 values per thread (the sm.mass storage)
+static_assert(MU_SLOTS >= 16, "a thread stages up to 7 + 8 values");
+
+// Level-0 bucket of s as an int and as a float (the same floor as bin0).
+__device__ __forceinline__ int bin0_both(float s, float m, float& bf) {
+  const float f = fminf(fmaxf((m - s) * BIN_SCALE, 0.0f), (float)(NB - 1));
+  const float fl = __fadd_rd(f, 8388608.0f);
+  bf = fl - 8388608.0f;
+  return __float_as_int(fl) - 0x4B000000;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <bool VEC>
 __device__ __noinline__ void mu_pass(RSmem& sm, const float* __restrict__ x, int V, float m,
                                      int g_lo, int g_hi, bool ent, MuPass& out) {
   constexpr int E = 8;
+  constexpr float kL = 1.4426950408889634f / 128.0f;  // log2(e) / 128
   const double md = (double)m;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* stage = reinterpret_cast<float*>(sm.mass) + warp * MU_STAGE;
-  unsigned long long* wbuf = sm.cand + warp * WCAP;
-  int sfill = 0, wfill = 0;  // warp-uniform fill levels
-  double mass = 0.0, qx = 0.0, rest = 0.0;
-  int cnt = 0;
+  const int tid = (int)threadIdx.x;
+  float* stage = reinterpret_cast<float*>(sm.mass) + tid;  // slot j at stage[j RT]
+  unsigned long long* tbuf = sm.cand + tid;
+  int sf = 0, tfill = 0, cnt = 0;
+  double mass = 0.0, qx = 0.0;
+  float rest = 0.0f;
   const unsigned gs = (unsigned)g_lo, gn = (unsigned)(g_hi - g_lo);
 
-  // weigh `n` staged values (n <= 8 * 32, lane j takes j, j + 32, ...)
+  // weigh this thread's first n <= 8 staged values
   auto weigh = [&](int n) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int i = e * 32 + lane;
-      if (i < n) {
-        const float s = stage[i];
-        const int b = bin0(s, m);
-        const double q = qmass_b(sm.tab, s, md, b);
+    for (int j = 0; j < E; ++j)
+      if (j < n) {
+        const float s = stage[j * RT];
+        const double q = qmass_b(sm.tab, s, md, bin0(s, m));
         mass += q;
         if (ent) qx += q * ((double)s - md);
       }
-    }
   };
 
   auto batch = [&](auto full, const float (&sv)[E], int a0, int na, int b0, int nb) {
     auto idx = [&](int e) { return e < 4 ? a0 + e : b0 + (e - 4); };
     auto ok = [&](int e) { return decltype(full)::value || (e < 4 ? e < na : e - 4 < nb); };
-    unsigned pre = 0, gm = 0;
+    unsigned gm = 0;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      const int b = bin0(sv[e], m);
+      float bf;
+      const int b = bin0_both(sv[e], m, bf);
       const bool v = ok(e);
-      pre |= (v && b < g_lo) ? 1u << e : 0u;
+      if (v && b < g_lo) {
+        stage[sf * RT] = sv[e];
+        ++sf;
+      }
       gm |= (v && (unsigned)b - gs <= gn) ? 1u << e : 0u;
-      if (v && b > g_hi) rest += tab_at(sm.tab, b);
+      if (v && b > g_hi) rest += ex2_approx(-(bf + 1.0f) * kL);
     }
-    cnt += __popc(pre);
-    // stage the kept values: one slot range per thread from a warp scan
-    {
-      const int c = __popc(pre);
-      int incl = c;
+    if (__any_sync(0xffffffffu, sf >= E)) {  // weigh eight, keep the rest staged
+      const int n = min(sf, E);
+      cnt += n;
+      weigh(n);
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int slot = sfill + incl - c;
-      sfill += __shfl_sync(0xffffffffu, incl, 31);
-#pragma unroll
-      for (int e = 0; e < E; ++e)
-        if ((pre >> e) & 1u) stage[slot++] = sv[e];
-      __syncwarp();
-      if (sfill >= 8 * 32) {  // a full batch: weigh it, move the rest to the front
-        weigh(8 * 32);
-        const int left = sfill - 8 * 32;  // < 8 * 32
-        float keep[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int i = e * 32 + lane;
-          keep[e] = i < left ? stage[8 * 32 + i] : 0.f;
-        }
-        __syncwarp();
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int i = e * 32 + lane;
-          if (i < left) stage[i] = keep[e];
-        }
-        __syncwarp();
-        sfill = left;
-      }
+      for (int j = 0; j < E - 1; ++j)
+        if (j + E < sf) stage[j * RT] = stage[(j + E) * RT];
+      sf -= n;
     }
     if (__any_sync(0xffffffffu, gm != 0u)) {
-      const int c = __popc(gm);
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int slot = wfill + incl - c;
-      wfill += __shfl_sync(0xffffffffu, incl, 31);
 #pragma unroll
       for (int e = 0; e < E; ++e)
         if ((gm >> e) & 1u) {
-          if (slot < WCAP) wbuf[slot] = ckey(sv[e], idx(e));
-          ++slot;
+          if (tfill < TCAP) tbuf[tfill * RT] = ckey(sv[e], idx(e));
+          ++tfill;
         }
     }
   };
 
-  const int tid = (int)threadIdx.x;
   int tail0 = 0;
   if (VEC) {
     const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
@@ -1363,18 +1330,21 @@ __device__ __noinline__ void mu_pass(RSmem& sm, const float* __restrict__ x, int
     const float sv[E] = {a, a, a, a, b, b, b, b};
     batch(std::false_type{}, sv, ia, ia < V ? 1 : 0, ib, ib < V ? 1 : 0);
   }
-  weigh(sfill);  // the last partial batch
-  if (lane == 0) sm.wcount[warp] = wfill;
-  double sums[4] = {mass, qx, rest, (double)cnt};  // counts are exact in a double
+  {  // the values still staged (at most E - 1 after the last batch)
+    const int n = min(sf, E);
+    cnt += n;
+    weigh(n);
+  }
+  sm.tcount[tid] = tfill;
+  // each fp32 term is within 2^-22 of its value and a thread sums a few hundred:
+  // 1e-4 covers both roundings, so the bound stays a lower bound
+  double sums[4] = {mass, qx, (double)rest * (1.0 - 1e-4), (double)cnt};
   block_sum_multi<4>(sums, sm);
   out.mass = sums[0];
   out.qx = sums[1];
-  out.rest_upper = sums[2];
+  out.rest_lower = sums[2];
   out.cnt = (long long)sums[3];
-  int ovf = 0;
-  for (int w = 0; w < NWARP; ++w) ovf |= sm.wcount[w] > WCAP ? 1 : 0;
-  out.overflow = ovf != 0;
-  __syncthreads();
+  out.overflow = __syncthreads_or(tfill > TCAP) != 0;
 }
 
 // Packs the live keys of the per-warp slices densely, in slice order, into the
@@ -1387,15 +1357,13 @@ __device__ __forceinline__ unsigned long long* packed(RSmem& sm) {
 
 __device__ __noinline__ int pack_gathered(RSmem& sm) {
   unsigned long long* g = packed(sm);
-  int off = 0;
-  for (int w = 0; w < NWARP; ++w) {
-    const int cnt = min(sm.wcount[w], WCAP);
-    for (int j = threadIdx.x; j < cnt; j += RT)
-      if (off + j < SCAP) g[off + j] = sm.cand[w * WCAP + j];
-    off += cnt;
-  }
+  const int mine = min(sm.tcount[threadIdx.x], TCAP);
+  long long tot;
+  const int off = (int)block_exscan<long long>((long long)mine, sm.red_l, tot);
+  for (int j = 0; j < mine; ++j)
+    if (off + j < SCAP) g[off + j] = sm.cand[j * RT + threadIdx.x];
   __syncthreads();
-  return min(off, SCAP);
+  return (int)min(tot, (long long)SCAP);
 }
 
 // Move the n packed candidates whose bucket lies in [lo, hi] to
@@ -1936,15 +1904,12 @@ __device__ int sampled_before(RSmem& sm, int b) {
   return r < 0 ? 0 : r;
 }
 
-// Applies f to every key left in the per-warp gather slices of pass 2 (each
-// slice holds at most WCAP = RT keys, so a thread visits one key per slice).
+// Applies f to every key this thread gathered in the pass before (its own
+// slots; together the threads visit every gathered key once).
 template <typename F>
 __device__ __forceinline__ void for_each_gathered(RSmem& sm, F&& f) {
-  static_assert(WCAP <= RT, "one key per thread per slice");
-  for (int w = 0; w < NWARP; ++w) {
-    const int cnt = min(sm.wcount[w], WCAP);
-    if ((int)threadIdx.x < cnt) f(sm.cand[w * WCAP + threadIdx.x]);
-  }
+  const int n = min(sm.tcount[threadIdx.x], TCAP);
+  for (int j = 0; j < n; ++j) f(sm.cand[j * RT + threadIdx.x]);
 }
 
 // Mass, count and smallest key of the gathered elements with key >= kt whose
@@ -2047,12 +2012,10 @@ __device__ __noinline__ bool resolve_row_planned(RSmem& sm, const float* __restr
   gathered_kept(sm, m, g2lo, bm, kt, km, kc, kmin, kx);
   if (kc == 0) return false;
   const Cut cm{kmin, mp.cnt + kc, mp.mass + km, mp.qx + kx};
-  // With top-p on, the min-p prefix decides when its mass stays below p Z.
-  // Each element after the gathered range weighs at least tab[b] exp(-1/128)
-  // (less 1e-5 for the fp32 rounding of its bucket index), so
-  // Z >= (its mass) + that bound, which certifies it; otherwise the fast path.
-  const double rest_lower = mp.rest_upper * exp(-1.0 / 128.0) * (1.0 - 1e-5);
-  if (p_on && !(cm.mass < (double)p * (cm.mass + rest_lower))) return false;
+  // With top-p on, the min-p prefix decides when its mass stays below p Z;
+  // Z >= (its mass) + the lower bound of the dropped elements' mass
+  // certifies it (otherwise the fast path decides).
+  if (p_on && !(cm.mass < (double)p * (cm.mass + mp.rest_lower))) return false;
   best = cm;
   return true;
 }
