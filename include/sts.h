@@ -170,6 +170,49 @@ sts_status sts_backward_sliced(const sts_shape* shape, const void* H_bf16, const
                                void* ws, size_t ws_bytes, sts_stream_t stream,
                                sts_slice_fn on_dw_slice, void* user, int comm_sms);
 
+/* Vocabulary-parallel tensor parallelism ("What this PR does", item 2 of the
+ * xorl PR: chunk-local logits gathered in rank order, hidden gradients summed
+ * across vocabulary ranks, weight-shard gradients kept local). Rank k holds
+ * the vocabulary rows [k Vl, (k + 1) Vl) of W. Each rank forms its shard's
+ * scaled logits (sts_scaled_logits), the ranks all-gather them, and
+ * sts_gather_vocab_shards interleaves the gathered blocks into full rows;
+ * every rank then runs the support program on the full rows
+ * (sts_resolve_logits) and the backward on its own shard
+ * (sts_backward_shard), whose partial dH the ranks sum. */
+
+/* dst[r * ld + k * vocab_per_rank + j] = src[(k * T + r) * vocab_per_rank + j]
+ * for k < world, r < T, j < vocab_per_rank: the world blocks [T, vocab_per_rank]
+ * of an all-gather, in rank order, into rows of stride ld >= world *
+ * vocab_per_rank. Device pointers (dst holds T * ld floats); asynchronous;
+ * allocates nothing. STS_ERR_SHAPE for non-positive sizes or a short ld. */
+sts_status sts_gather_vocab_shards(const float* src, int64_t world, int64_t T,
+                                   int64_t vocab_per_rank, float* dst, int64_t ld,
+                                   sts_stream_t stream);
+
+/* The forward's support program, logprob and saved scalars (and optionally
+ * the entropy) on caller-given fp32 scaled logits S [T, ld] (row stride ld >=
+ * shape->V; the first V columns of each row are the row), for example full
+ * rows gathered from vocabulary shards. The row max is taken from S. Rows are
+ * validated as in sts_forward (temperature included: the backward divides by
+ * it). ws: sts_workspace_bytes(shape, 2). saved->flags doubles as the row
+ * flags. */
+sts_status sts_resolve_logits(const sts_shape* shape, const float* S, int64_t ld,
+                              const sts_rows* rows, float* logprob, float* entropy,
+                              const sts_saved* saved, void* ws, size_t ws_bytes,
+                              sts_stream_t stream);
+
+/* The backward of one rank's vocabulary shard: W_shard holds the vocabulary
+ * rows [vocab_offset, vocab_offset + shape->V) of the full W, rows->target and
+ * the saved scalars (cut ids) use full-vocabulary ids. Writes dW_shard
+ * [shape->V, d] (overwritten unless accumulate_dW) and dH_partial [T, d] =
+ * this shard's part of dH, which the ranks sum. ws: sts_workspace_bytes(shape,
+ * 1). STS_ERR_SHAPE for a negative offset. */
+sts_status sts_backward_shard(const sts_shape* shape, const void* H_bf16, const void* W_shard_bf16,
+                              const sts_rows* rows, const sts_saved* saved,
+                              const float* grad_logprob, float* dH_partial, float* dW_shard,
+                              int accumulate_dW, int64_t vocab_offset, void* ws, size_t ws_bytes,
+                              sts_stream_t stream);
+
 /* Draw one token per row from the filtered distribution: the inverse CDF of
  * the support walked in (s desc, id asc) order, taking the first kept token
  * whose inclusive running mass exceeds u[t] * sum_{i in S} exp(s_i - m).

@@ -22,6 +22,7 @@ import os
 import torch
 
 from .dp import SliceAllReduce  # noqa: E402
+from .tp import VocabParallel  # noqa: E402
 
 __all__ = [
     "StsError",
@@ -31,6 +32,10 @@ __all__ = [
     "sts_vocab_chunk",
     "sts_forward",
     "sts_backward",
+    "sts_backward_shard",
+    "sts_resolve_logits",
+    "sts_gather_vocab_shards",
+    "VocabParallel",
     "SliceAllReduce",
     "sts_sample",
     "sts_filter_logits",
@@ -84,6 +89,9 @@ EXPORTED_SYMBOLS = (
     "sts_policy_grad",
     "sts_path_counts",
     "sts_backward_sliced",
+    "sts_backward_shard",
+    "sts_resolve_logits",
+    "sts_gather_vocab_shards",
 )
 
 
@@ -146,6 +154,14 @@ def load():
                                         ctypes.POINTER(_Saved), P, P, P, ctypes.c_int, P, S, P,
                                         _SLICE_FN, P, ctypes.c_int]
     lib.sts_backward_sliced.restype = ctypes.c_int
+    lib.sts_backward_shard.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows),
+                                       ctypes.POINTER(_Saved), P, P, P, ctypes.c_int, I64, P, S, P]
+    lib.sts_backward_shard.restype = ctypes.c_int
+    lib.sts_resolve_logits.argtypes = [ctypes.POINTER(_Shape), P, I64, ctypes.POINTER(_Rows), P, P,
+                                       ctypes.POINTER(_Saved), P, S, P]
+    lib.sts_resolve_logits.restype = ctypes.c_int
+    lib.sts_gather_vocab_shards.argtypes = [P, I64, I64, I64, P, I64, P]
+    lib.sts_gather_vocab_shards.restype = ctypes.c_int
     lib.sts_sample.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows), P, P, P, S, P]
     lib.sts_sample.restype = ctypes.c_int
     lib.sts_filter_logits.argtypes = [ctypes.POINTER(_Shape), P, ctypes.POINTER(_Rows), P, P, P, P,
@@ -532,3 +548,85 @@ def sts_path_counts(ws, stream=None):
     counts = (ctypes.c_int64 * 4)()
     _check(lib.sts_path_counts(_ptr(ws), _stream(stream), counts), "sts_path_counts")
     return {name: int(counts[i]) for i, name in enumerate(RESOLVE_PATHS)}
+
+
+def _saved_tensors(T, dev):
+    return {
+        "row_max": torch.empty(T, dtype=torch.float32, device=dev),
+        "lse_support": torch.empty(T, dtype=torch.float32, device=dev),
+        "cut_logit": torch.empty(T, dtype=torch.float32, device=dev),
+        "cut_id": torch.empty(T, dtype=torch.int32, device=dev),
+        "support_size": torch.empty(T, dtype=torch.int32, device=dev),
+        "flags": torch.empty(T, dtype=torch.int32, device=dev),
+    }
+
+
+def _saved_struct(saved):
+    return _Saved(*(_ptr(saved[k]) for k in ("row_max", "lse_support", "cut_logit", "cut_id",
+                                              "support_size", "flags")))
+
+
+def sts_resolve_logits(S, target, temperature, top_k, top_p, min_p, *, V=None, entropy=False,
+                       ws=None, stream=None, check=False):
+    """The support program, logprob and saved scalars on fp32 scaled logits
+    S [T, ld] (the first V columns of each row; V defaults to ld)."""
+    lib = load()
+    _need(S, torch.float32, "S")
+    T, ld = S.shape
+    V = ld if V is None else int(V)
+    rows = _rows(T, target, temperature, top_k, top_p, min_p)
+    sh = _shape(T, 8, V)
+    ws = _workspace(sts_workspace_bytes(T, 8, V, 2), S.device, ws)
+    logprob = torch.empty(T, dtype=torch.float32, device=S.device)
+    saved = _saved_tensors(T, S.device)
+    ent = torch.empty(T, dtype=torch.float32, device=S.device) if entropy else None
+    st = lib.sts_resolve_logits(ctypes.byref(sh), _ptr(S), ld, ctypes.byref(rows), _ptr(logprob),
+                                _ptr(ent), ctypes.byref(_saved_struct(saved)), _ptr(ws), ws.numel(),
+                                _stream(stream))
+    _check(st, "sts_resolve_logits")
+    if ent is not None:
+        saved["entropy"] = ent
+    if check:
+        sts_get_status(ws, stream, raise_on_error=True)
+    return logprob, saved, ws
+
+
+def sts_backward_shard(H, W_shard, target, temperature, top_k, top_p, min_p, saved, grad_logprob,
+                       *, vocab_offset, dW=None, dH=None, accumulate_dW=False, vocab_chunk=0,
+                       ws=None, stream=None, check=False):
+    """One vocabulary shard's backward: (dH_partial [T, d], dW_shard [Vl, d])."""
+    lib = load()
+    T, d, Vl = _hw(H, W_shard)
+    rows = _rows(T, target, temperature, top_k, top_p, min_p)
+    _need(grad_logprob, torch.float32, "grad_logprob", (T,))
+    sh = _shape(T, d, Vl, vocab_chunk, 0)
+    dev = H.device
+    ws = _workspace(sts_workspace_bytes(T, d, Vl, 1, vocab_chunk, 0), dev, ws)
+    dH = torch.empty((T, d), dtype=torch.float32, device=dev) if dH is None else dH
+    if dW is None:
+        if accumulate_dW:
+            raise StsError(STS_ERR_NULL, "accumulate_dW needs a dW tensor")
+        dW = torch.empty((Vl, d), dtype=torch.float32, device=dev)
+    _need(dH, torch.float32, "dH", (T, d))
+    _need(dW, torch.float32, "dW", (Vl, d))
+    st = lib.sts_backward_shard(ctypes.byref(sh), _ptr(H), _ptr(W_shard), ctypes.byref(rows),
+                                ctypes.byref(_saved_struct(saved)), _ptr(grad_logprob), _ptr(dH),
+                                _ptr(dW), 1 if accumulate_dW else 0, int(vocab_offset), _ptr(ws),
+                                ws.numel(), _stream(stream))
+    _check(st, "sts_backward_shard")
+    if check:
+        sts_get_status(ws, stream, raise_on_error=True)
+    return dH, dW
+
+
+def sts_gather_vocab_shards(src, dst, *, stream=None):
+    """dst [T, ld] <- the rank-order interleave of src [world, T, Vl]."""
+    lib = load()
+    _need(src, torch.float32, "src")
+    _need(dst, torch.float32, "dst")
+    world, T, Vl = src.shape
+    if dst.shape[0] != T:
+        raise StsError(STS_ERR_SHAPE, "dst rows must equal the shards' rows")
+    _check(lib.sts_gather_vocab_shards(_ptr(src), world, T, Vl, _ptr(dst), dst.shape[1],
+                                       _stream(stream)), "sts_gather_vocab_shards")
+    return dst

@@ -17,7 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsts.so")
-SOURCES = ["sts_api.cu", "resolver.cu", "noalloc.cu", "policy.cu"]
+SOURCES = ["sts_api.cu", "resolver.cu", "noalloc.cu", "policy.cu", "tp.cu"]
 HEADERS = ["sts_device.cuh", "gemm_sm100.cuh", "sts_internal.h"]
 
 

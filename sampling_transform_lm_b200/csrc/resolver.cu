@@ -108,7 +108,8 @@ struct RSmem {
   // copies (one thread issues them, chunks in flight = NSTAGE).
   float4 ring[NSTAGE][CH_F4];
   unsigned long long full_bar[NSTAGE];   // bulk copy landed (tx bytes)
-  unsigned long long empty_bar[NSTAGE];  // every warp done with the chunk
+  int ring_done[NSTAGE];                 // warps done with the chunk in the slot
+  int ring_issued;                       // copies issued in the current pass
   int abort_flag;                        // a bounded wait gave up
   uint32_t ring_q[RT];                   // per thread: chunks consumed so far (all equal)
   int* err;                              // the workspace status word's error field
@@ -275,10 +276,10 @@ __device__ __forceinline__ void for_each(const float* __restrict__ x, int V, F&&
 // ---------------------------------------------------------------- streaming through the ring
 // A row whose start is 16-byte aligned is read in chunks of CH_F4 float4s
 // (chunk c = float4s [c CH_F4, min(V4, (c + 1) CH_F4))) that bulk copies put
-// into the shared-memory ring. Thread 0 keeps up to NSTAGE copies in flight, so
-// a pass's HBM latency is covered without holding loads in registers; every
-// thread takes the float4s at offsets t and t + RT of each chunk and each warp
-// releases a chunk when its lanes are done with it.
+// into the shared-memory ring. Up to NSTAGE copies are in flight, so a pass's
+// HBM latency is covered without holding loads in registers; every thread
+// takes the float4s at offsets t and t + RT of each chunk, and the warp that
+// finishes a chunk last copies the chunk NSTAGE ahead into its slot.
 //
 // stream_chunks streams chunks chunk_of(0), ..., chunk_of(n - 1) and calls
 // f(full, a, ia, b, ib, va, vb) for each: a and b the thread's two float4s,
@@ -297,25 +298,23 @@ __device__ __forceinline__ bool stream_chunks(RSmem& sm, const float4* __restric
   const int tid = (int)threadIdx.x, lane = tid & 31;
   volatile int* abort_flag = &sm.abort_flag;
   const uint32_t q0 = sm.ring_q[tid];
-  int issued = 0;  // thread 0
-  auto issue = [&](int j) -> bool {
+  // copy chunk j into its slot (the slot's previous chunk is fully consumed)
+  auto issue = [&](int j) {
     const uint32_t qq = q0 + (uint32_t)j;
     const int s = (int)(qq % NSTAGE);
-    if (qq >= (uint32_t)NSTAGE &&
-        !mbar_wait(smem_u32(&sm.empty_bar[s]), ((qq / NSTAGE) - 1u) & 1u, abort_flag, err))
-      return false;
     const int f0 = chunk_of(j) * CH_F4;
     const uint32_t bytes = (uint32_t)min(CH_F4, V4 - f0) * 16u;
     mbar_arrive_expect_tx(smem_u32(&sm.full_bar[s]), bytes);
     bulk_load(smem_u32(&sm.ring[s][0]), x4 + f0, bytes, smem_u32(&sm.full_bar[s]), policy);
-    ++issued;
-    return true;
+    atomicAdd(&sm.ring_issued, 1);
   };
+  if (tid == 0) {
+    sm.ring_issued = 0;
+    for (int j = 0; j < n && j < NSTAGE; ++j) issue(j);
+  }
   bool ok = true;
-  if (tid == 0)
-    for (int j = 0; j < n && j < NSTAGE && ok; ++j) ok = issue(j);
   int j = 0;
-  for (; j < n && ok; ++j) {
+  for (; j < n; ++j) {
     const uint32_t qq = q0 + (uint32_t)j;
     const int s = (int)(qq % NSTAGE);
     if (!mbar_wait(smem_u32(&sm.full_bar[s]), (qq / NSTAGE) & 1u, abort_flag, err)) {
@@ -331,19 +330,34 @@ __device__ __forceinline__ bool stream_chunks(RSmem& sm, const float4* __restric
     else
       f(std::false_type{}, a, f0 + tid, b, f0 + tid + RT, tid < cnt, tid + RT < cnt);
     __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&sm.empty_bar[s]));
-    if (tid == 0 && j + NSTAGE < n && ok) ok = issue(j + NSTAGE);
+    // the warp that finishes a chunk last refills its slot: no warp waits for
+    // another one to release a slot
+    if (lane == 0) {
+      __threadfence_block();
+      if (atomicAdd(&sm.ring_done[s], 1) == NWARP - 1) {
+        sm.ring_done[s] = 0;
+        if (j + NSTAGE < n) {
+          __threadfence_block();
+          fence_proxy_async_smem();  // every warp's reads of the slot before the copy
+          issue(j + NSTAGE);
+        }
+      }
+    }
   }
-  if (!ok) {
-    *abort_flag = 1;
-    if (tid == 0)  // copies issued but not consumed may still be landing
-      for (int k = j; k < issued; ++k) {
+  if (!ok) *abort_flag = 1;
+  sm.ring_q[tid] = q0 + (uint32_t)n;
+  // every slot consumed before the next pass fills it; on a failed wait,
+  // thread 0 waits (bounded) for the copies issued after its last chunk
+  if (__syncthreads_or(!ok)) {
+    if (tid == 0)
+      for (int k = j; k < sm.ring_issued; ++k) {
         const uint32_t qq = q0 + (uint32_t)k;
         mbar_wait_drain(smem_u32(&sm.full_bar[qq % NSTAGE]), (qq / NSTAGE) & 1u);
       }
+    __syncthreads();
+    return false;
   }
-  sm.ring_q[tid] = q0 + (uint32_t)n;
-  return ok;
+  return true;
 }
 
 // Number of chunks of a row of V4 float4s.
@@ -2031,7 +2045,7 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
     sm.bd[3] = exp(-1.0 / 256.0);  // mid-bucket weight factor
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(smem_u32(&sm.full_bar[s]), 1);
-      mbar_init(smem_u32(&sm.empty_bar[s]), NWARP);
+      sm.ring_done[s] = 0;
     }
     sm.abort_flag = 0;
     sm.err = &a.hdr->err;

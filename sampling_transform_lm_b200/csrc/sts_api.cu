@@ -355,6 +355,97 @@ sts_status forward_impl(const sts_shape* shape, const void* H, const void* W, co
   return STS_OK;
 }
 
+// The backward over W's vocabulary rows [0, V); their ids in the full
+// vocabulary start at vocab_offset (0 unless W is one rank's vocabulary shard).
+sts_status backward_impl(const sts_shape* shape, const void* H, const void* W,
+                         const sts_rows* rows, const sts_saved* saved, const float* grad,
+                         float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
+                         sts_stream_t stream, sts_slice_fn on_dw_slice, void* user, int comm_sms,
+                         int64_t vocab_offset) {
+  if (!shape_ok(shape)) return STS_ERR_SHAPE;
+  if (comm_sms < 0) return STS_ERR_SHAPE;
+  if (vocab_offset < 0 || vocab_offset + shape->V > (int64_t(1) << 31) - 1) return STS_ERR_SHAPE;
+  if (!H || !W || !grad || !dH || !dW) return STS_ERR_NULL;
+  STS_TRY(check_rows(shape, rows, true));
+  if (!saved || !saved->lse_support || !saved->cut_logit || !saved->cut_id || !saved->flags)
+    return STS_ERR_NULL;
+  if (!aligned16(H) || !aligned16(W) || !aligned16(dH) || !aligned16(dW)) return STS_ERR_SHAPE;
+  const BwdLayout L = bwd_layout(shape);
+  STS_TRY(check_ws(ws, ws_bytes, L.total));
+  DeviceInfo dev;
+  STS_TRY(device_info(dev));
+  if (comm_sms >= dev.sms) return STS_ERR_SHAPE;
+  dev.sms -= comm_sms;  // persistent GEMMs leave these SMs to the caller's exchange kernels
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  const int64_t T = shape->T, V = shape->V, d = shape->d, Vc = vocab_chunk(shape);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
+  void* dZ = wsb + L.dz_off;
+  STS_TRY(reset_header(ws, st));
+
+  CUtensorMap m_h_k, m_w_k, m_h_mn, m_w_mn, m_dw, m_dh;
+  if (!map_kmajor(&m_h_k, H, d, T, d, GEMM_BM) || !map_kmajor(&m_w_k, W, d, V, d, GEMM_BN) ||
+      !map_mnmajor(&m_h_mn, H, d, T, d) || !map_mnmajor(&m_w_mn, W, d, V, d) ||
+      !map_out_f32(&m_dw, dW, d, V, d) || !map_out_f32(&m_dh, dH, d, T, d))
+    return STS_ERR_CUDA;
+
+  for (int64_t v0 = 0; v0 < V; v0 += Vc) {
+    const int64_t w = (V - v0) < Vc ? (V - v0) : Vc;
+    CUtensorMap m_dz_out, m_dz_k, m_dz_mn;
+    if (!map_out_bf16(&m_dz_out, dZ, w, T, Vc) || !map_kmajor(&m_dz_k, dZ, w, T, Vc, GEMM_BM) ||
+        !map_mnmajor(&m_dz_mn, dZ, w, T, Vc))
+      return STS_ERR_CUDA;
+
+    // 1. recompute the chunk's logits and form dZ in the epilogue
+    GemmParams p{};
+    p.M = (int)T;
+    p.N = (int)w;
+    p.K = (int)d;
+    p.b_mn0 = (int)v0;
+    p.tau = rows->temperature;
+    p.lse = saved->lse_support;
+    p.cut_logit = saved->cut_logit;
+    p.cut_id = saved->cut_id;
+    p.target = rows->target;
+    p.grad = grad;
+    p.flags = saved->flags;
+    p.col_base = (int)(vocab_offset + v0);
+    p.err = &hdr->err;
+    STS_CUDA(timed_launch(STS_KERNEL_DZ_GEMM, st, [&] {
+      return run_gemm<false, false, kEpiDZ>(m_h_k, m_w_k, m_dz_out, p, dev.sms, st);
+    }));
+
+    // 2. dW[v0:v0+w] = dZ^T . H (both operands MN-major), written once
+    GemmParams q{};
+    q.M = (int)w;
+    q.N = (int)d;
+    q.K = (int)T;
+    q.c_y0 = (int)v0;
+    q.err = &hdr->err;
+    STS_CUDA(timed_launch(STS_KERNEL_DW_GEMM, st, [&] {
+      return accumulate_dW ? run_gemm<true, true, kEpiReduceF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st)
+                           : run_gemm<true, true, kEpiStoreF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st);
+    }));
+    // the slice is final once this GEMM completes on `st`: hand it out before
+    // enqueuing the work that follows, so its exchange overlaps that work
+    if (on_dw_slice) on_dw_slice(user, v0, w, dW + (size_t)v0 * (size_t)d, stream);
+
+    // 3. dH (+)= dZ . W[v0:v0+w] (W read MN-major)
+    GemmParams r{};
+    r.M = (int)T;
+    r.N = (int)d;
+    r.K = (int)w;
+    r.b_k0 = (int)v0;
+    r.err = &hdr->err;
+    STS_CUDA(timed_launch(STS_KERNEL_DH_GEMM, st, [&] {
+      return v0 == 0 ? run_gemm<false, true, kEpiStoreF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st)
+                     : run_gemm<false, true, kEpiReduceF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st);
+    }));
+  }
+  return STS_OK;
+}
+
 }  // namespace
 }  // namespace sts
 
@@ -419,94 +510,70 @@ sts_status sts_backward_sliced(const sts_shape* shape, const void* H, const void
                                float* dH, float* dW, int accumulate_dW, void* ws, size_t ws_bytes,
                                sts_stream_t stream, sts_slice_fn on_dw_slice, void* user,
                                int comm_sms) {
-  if (!shape_ok(shape)) return STS_ERR_SHAPE;
-  if (comm_sms < 0) return STS_ERR_SHAPE;
-  if (!H || !W || !grad || !dH || !dW) return STS_ERR_NULL;
-  STS_TRY(check_rows(shape, rows, true));
-  if (!saved || !saved->lse_support || !saved->cut_logit || !saved->cut_id || !saved->flags)
-    return STS_ERR_NULL;
-  if (!aligned16(H) || !aligned16(W) || !aligned16(dH) || !aligned16(dW)) return STS_ERR_SHAPE;
-  const BwdLayout L = bwd_layout(shape);
-  STS_TRY(check_ws(ws, ws_bytes, L.total));
-  DeviceInfo dev;
-  STS_TRY(device_info(dev));
-  if (comm_sms >= dev.sms) return STS_ERR_SHAPE;
-  dev.sms -= comm_sms;  // persistent GEMMs leave these SMs to the caller's exchange kernels
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-
-  const int64_t T = shape->T, V = shape->V, d = shape->d, Vc = vocab_chunk(shape);
-  uint8_t* wsb = static_cast<uint8_t*>(ws);
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(wsb);
-  void* dZ = wsb + L.dz_off;
-  STS_TRY(reset_header(ws, st));
-
-  CUtensorMap m_h_k, m_w_k, m_h_mn, m_w_mn, m_dw, m_dh;
-  if (!map_kmajor(&m_h_k, H, d, T, d, GEMM_BM) || !map_kmajor(&m_w_k, W, d, V, d, GEMM_BN) ||
-      !map_mnmajor(&m_h_mn, H, d, T, d) || !map_mnmajor(&m_w_mn, W, d, V, d) ||
-      !map_out_f32(&m_dw, dW, d, V, d) || !map_out_f32(&m_dh, dH, d, T, d))
-    return STS_ERR_CUDA;
-
-  for (int64_t v0 = 0; v0 < V; v0 += Vc) {
-    const int64_t w = (V - v0) < Vc ? (V - v0) : Vc;
-    CUtensorMap m_dz_out, m_dz_k, m_dz_mn;
-    if (!map_out_bf16(&m_dz_out, dZ, w, T, Vc) || !map_kmajor(&m_dz_k, dZ, w, T, Vc, GEMM_BM) ||
-        !map_mnmajor(&m_dz_mn, dZ, w, T, Vc))
-      return STS_ERR_CUDA;
-
-    // 1. recompute the chunk's logits and form dZ in the epilogue
-    GemmParams p{};
-    p.M = (int)T;
-    p.N = (int)w;
-    p.K = (int)d;
-    p.b_mn0 = (int)v0;
-    p.tau = rows->temperature;
-    p.lse = saved->lse_support;
-    p.cut_logit = saved->cut_logit;
-    p.cut_id = saved->cut_id;
-    p.target = rows->target;
-    p.grad = grad;
-    p.flags = saved->flags;
-    p.col_base = (int)v0;
-    p.err = &hdr->err;
-    STS_CUDA(timed_launch(STS_KERNEL_DZ_GEMM, st, [&] {
-      return run_gemm<false, false, kEpiDZ>(m_h_k, m_w_k, m_dz_out, p, dev.sms, st);
-    }));
-
-    // 2. dW[v0:v0+w] = dZ^T . H (both operands MN-major), written once
-    GemmParams q{};
-    q.M = (int)w;
-    q.N = (int)d;
-    q.K = (int)T;
-    q.c_y0 = (int)v0;
-    q.err = &hdr->err;
-    STS_CUDA(timed_launch(STS_KERNEL_DW_GEMM, st, [&] {
-      return accumulate_dW ? run_gemm<true, true, kEpiReduceF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st)
-                           : run_gemm<true, true, kEpiStoreF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st);
-    }));
-    // the slice is final once this GEMM completes on `st`: hand it out before
-    // enqueuing the work that follows, so its exchange overlaps that work
-    if (on_dw_slice) on_dw_slice(user, v0, w, dW + (size_t)v0 * (size_t)d, stream);
-
-    // 3. dH (+)= dZ . W[v0:v0+w] (W read MN-major)
-    GemmParams r{};
-    r.M = (int)T;
-    r.N = (int)d;
-    r.K = (int)w;
-    r.b_k0 = (int)v0;
-    r.err = &hdr->err;
-    STS_CUDA(timed_launch(STS_KERNEL_DH_GEMM, st, [&] {
-      return v0 == 0 ? run_gemm<false, true, kEpiStoreF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st)
-                     : run_gemm<false, true, kEpiReduceF32>(m_dz_k, m_w_mn, m_dh, r, dev.sms, st);
-    }));
-  }
-  return STS_OK;
+  return backward_impl(shape, H, W, rows, saved, grad, dH, dW, accumulate_dW, ws, ws_bytes, stream,
+                       on_dw_slice, user, comm_sms, 0);
 }
 
 sts_status sts_backward(const sts_shape* shape, const void* H, const void* W, const sts_rows* rows,
                         const sts_saved* saved, const float* grad, float* dH, float* dW,
                         int accumulate_dW, void* ws, size_t ws_bytes, sts_stream_t stream) {
-  return sts_backward_sliced(shape, H, W, rows, saved, grad, dH, dW, accumulate_dW, ws, ws_bytes,
-                             stream, nullptr, nullptr, 0);
+  return backward_impl(shape, H, W, rows, saved, grad, dH, dW, accumulate_dW, ws, ws_bytes, stream,
+                       nullptr, nullptr, 0, 0);
+}
+
+sts_status sts_backward_shard(const sts_shape* shape, const void* H, const void* W_shard,
+                              const sts_rows* rows, const sts_saved* saved, const float* grad,
+                              float* dH_partial, float* dW_shard, int accumulate_dW,
+                              int64_t vocab_offset, void* ws, size_t ws_bytes, sts_stream_t stream) {
+  return backward_impl(shape, H, W_shard, rows, saved, grad, dH_partial, dW_shard, accumulate_dW, ws,
+                       ws_bytes, stream, nullptr, nullptr, 0, vocab_offset);
+}
+
+sts_status sts_resolve_logits(const sts_shape* shape, const float* S, int64_t ld,
+                              const sts_rows* rows, float* logprob, float* entropy,
+                              const sts_saved* saved, void* ws, size_t ws_bytes,
+                              sts_stream_t stream) {
+  if (!shape_ok(shape)) return STS_ERR_SHAPE;
+  if (!S || !logprob) return STS_ERR_NULL;
+  if (ld < shape->V) return STS_ERR_SHAPE;
+  STS_TRY(check_rows(shape, rows, true));
+  if (!saved || !saved->row_max || !saved->lse_support || !saved->cut_logit || !saved->cut_id ||
+      !saved->support_size || !saved->flags)
+    return STS_ERR_NULL;
+  STS_TRY(check_ws(ws, ws_bytes, filter_bytes(shape)));
+  DeviceInfo dev;
+  STS_TRY(device_info(dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  int32_t* flags = saved->flags;
+  STS_TRY(reset_header(ws, st));
+  STS_CUDA(timed_launch(STS_KERNEL_VALIDATE, st, [&] {
+    launch_validate(rows->target, rows->temperature, rows->top_p, rows->min_p, shape->T, shape->V,
+                    flags, hdr, true, st);
+    return cudaGetLastError();
+  }));
+  ResolveArgs a{};
+  a.S = S;
+  a.ld = ld;
+  a.rows = (int)shape->T;
+  a.V = (int)shape->V;
+  a.mode = kModeForward;
+  a.target = rows->target;
+  a.top_k = rows->top_k;
+  a.top_p = rows->top_p;
+  a.min_p = rows->min_p;
+  a.row_flags = flags;
+  a.flags_out = flags;
+  a.logprob = logprob;
+  a.entropy = entropy;
+  a.row_max = saved->row_max;
+  a.lse_support = saved->lse_support;
+  a.cut_logit = saved->cut_logit;
+  a.cut_id = saved->cut_id;
+  a.support_size = saved->support_size;
+  a.hdr = hdr;
+  STS_CUDA(timed_launch(STS_KERNEL_RESOLVE, st, [&] { return launch_resolve(a, dev.sms, st); }));
+  return STS_OK;
 }
 
 sts_status sts_filter_logits(const sts_shape* shape, const float* S, const sts_rows* rows,

@@ -3,6 +3,7 @@ float64 oracle, through the C ABI, on seeded inputs that span several tiles
 and ragged tails, plus the edge cases of the method."""
 
 import math
+import socket
 
 import numpy as np
 import pytest
@@ -347,3 +348,73 @@ def test_sliced_backward_allreduce_single_rank(cuda_lib):
         dist.destroy_process_group()
     assert order == [(v0, min(512, 2500 - v0)) for v0 in range(0, 2500, 512)]
     assert torch.equal(dW1, dW0) and torch.equal(dH1, dH0)
+
+
+def test_vocab_shards_reproduce_the_unsharded_path(cuda_lib):
+    """Two vocabulary shards on one GPU, without collectives: the shards'
+    logits (sts_scaled_logits) interleaved in rank order by
+    sts_gather_vocab_shards equal the full projection bit for bit, the support
+    program on them (sts_resolve_logits) gives sts_forward's logprob and saved
+    scalars bit for bit, each shard's backward (sts_backward_shard) gives its
+    rows of dW bit for bit, and the two partial dH add up to dH."""
+    sts = cuda_lib
+    T, d, V = 260, 136, 2 * 1280
+    H, W, meta, u = small_case(23, T, d, V)
+    Hf, Wf, s, rows = _oracle_case(H, W, meta, u)
+    Hd, Wd = bf16_tensor(H), bf16_tensor(W)
+    y, tau, k, p, mu = row_tensors(rows)
+    lp0, saved0, _ = sts.sts_forward(Hd, Wd, y, tau, k, p, mu, check=True, entropy=True)
+    g = torch.from_numpy(np.asarray(workloads.extra_grad(23, T))).cuda()
+    dH0, dW0 = sts.sts_backward(Hd, Wd, y, tau, k, p, mu, saved0, g, vocab_chunk=512, check=True)
+    vl = V // 2
+    blocks = torch.stack([sts.sts_scaled_logits(Hd, Wd[r * vl:(r + 1) * vl].contiguous(), tau)
+                          for r in range(2)])
+    full = torch.empty((T, V), dtype=torch.float32, device="cuda")
+    sts.sts_gather_vocab_shards(blocks.contiguous(), full)
+    assert torch.equal(full, sts.sts_scaled_logits(Hd, Wd, tau))
+    lp1, saved1, _ = sts.sts_resolve_logits(full, y, tau, k, p, mu, check=True, entropy=True)
+    assert torch.equal(lp1, lp0)
+    for key in ("row_max", "lse_support", "cut_logit", "cut_id", "support_size", "flags",
+                "entropy"):
+        assert torch.equal(saved1[key], saved0[key]), key
+    parts = [sts.sts_backward_shard(Hd, Wd[r * vl:(r + 1) * vl].contiguous(), y, tau, k, p, mu,
+                                    saved1, g, vocab_offset=r * vl, vocab_chunk=512, check=True)
+             for r in range(2)]
+    assert torch.equal(torch.cat([parts[0][1], parts[1][1]]), dW0)
+    dH = parts[0][0] + parts[1][0]
+    assert rel_fro(dH.cpu().numpy(), dH0.cpu().numpy()) < 1e-6
+
+
+def test_vocab_parallel_single_rank_nccl(cuda_lib):
+    """VocabParallel over a one-rank NCCL group (the collectives are the
+    identity): the same logprobs, dH and dW as the unsharded path."""
+    import datetime
+
+    import torch.distributed as dist
+
+    from sampling_transform_lm_b200.tp import VocabParallel
+
+    sts = cuda_lib
+    T, d, V = 300, 64, 1024
+    H, W, meta, u = small_case(24, T, d, V)
+    Hf, Wf, s, rows = _oracle_case(H, W, meta, u)
+    Hd, Wd = bf16_tensor(H), bf16_tensor(W)
+    y, tau, k, p, mu = row_tensors(rows)
+    lp0, saved0, _ = sts.sts_forward(Hd, Wd, y, tau, k, p, mu, check=True)
+    g = torch.ones(T, dtype=torch.float32, device="cuda")
+    dH0, dW0 = sts.sts_backward(Hd, Wd, y, tau, k, p, mu, saved0, g, check=True)
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        tp = VocabParallel(row_chunk=128)
+        lp, saved = tp.forward(Hd, Wd, y, tau, k, p, mu)
+        dH, dW = tp.backward(Hd, Wd, y, tau, k, p, mu, saved, g)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    assert torch.equal(lp, lp0) and torch.equal(dW, dW0) and torch.equal(dH, dH0)
