@@ -33,7 +33,11 @@
 //                top-p is on too, only where the sample puts the crossing
 //                clearly after the min-p prefix). One pass gathers that range
 //                and, for min-p, weighs and counts everything before it, and
-//                the row is decided from the gathered elements.
+//                the row is decided from the gathered elements. Without the
+//                entropy output (and outside the sampler) a min-p-decided row
+//                is weighed in fp32 instead (kept iff s >= t; the support's
+//                mass only enters LSE_S and, with top-p on, a certificate
+//                checked against the fp32 error bound), as are identity rows.
 //   fast path    (rows whose plan does not hold, and top-p rows) a count pass
 //                adds the rest of the row to the sample's histogram; the top-p
 //                crossing's bucket is estimated from the counts with
@@ -45,7 +49,12 @@
 //                row's lines evict-last) forms float64 masses of every element,
 //                summed in registers (the total, the mass before the window, the
 //                mass before the min-p bucket), and gathers the planned buckets'
-//                elements into per-warp slices of a candidate buffer.
+//                elements into per-thread slots of a candidate buffer. A pass
+//                that only gathers (top-k) tests values against the planned
+//                buckets widened by one, without forming bucket indices.
+//   large top-k  (the prefix up to the k-th element's bucket exceeds the sort)
+//                one exact pass gathers that bucket alone; its sorted elements
+//                give the k-th element and Z_k.
 //   finish       exact masses of the window buckets place the crossing in one
 //                bucket; its elements are sorted by composite key (a bitonic
 //                network held mostly in registers and warp shuffles) and
@@ -55,8 +64,7 @@
 //                renormalised support: ln Z_S - sum_S q (s - m) / Z_S.
 //
 // When the plan cannot be proven to hold a cut (a crossing outside the
-// window, too many candidates, large top-k) the row falls back to the exact
-// search: a float64 mass histogram, then the candidate buckets gathered from
+// window, too many candidates) the row falls back to the exact search: a float64 mass histogram, then the candidate buckets gathered from
 // the row, refining a bucket too large for the 4096-entry sort on its
 // composite keys (12 bits per level) until it fits; the keys are distinct, so
 // this ends after at most six levels.
@@ -160,7 +168,9 @@ __device__ __forceinline__ int ckey_id(unsigned long long K) {
 // takes no conversion instruction: adding 2^23 rounding toward -inf leaves
 // floor(f) in the low mantissa bits (f < 2^23, one unit per ulp).
 __device__ __forceinline__ int bin0(float s, float m) {
-  const float f = fminf(fmaxf((m - s) * BIN_SCALE, 0.0f), (float)(NB - 1));
+  // fma(s, -128, 128 m) rounds 128 (m - s) once, which equals 128 fl(m - s):
+  // scaling by a power of two commutes with rounding
+  const float f = fminf(fmaxf(fmaf(s, -BIN_SCALE, m * BIN_SCALE), 0.0f), (float)(NB - 1));
   return __float_as_int(__fadd_rd(f, 8388608.0f)) - 0x4B000000;
 }
 
@@ -937,8 +947,8 @@ __device__ __noinline__ float row_max_pass(const float* __restrict__ x, int V) {
 
 // ---------------------------------------------------------------- exact path
 // Float64 mass histogram (atomics) and the general search: used when the fast
-// path below cannot prove its window holds the cut (large top-k, oversized
-// buckets, a crossing outside the estimated window).
+// path below cannot prove its window holds the cut (a bucket too large for
+// the sort, a crossing outside the estimated window).
 template <bool VEC>
 __device__ __noinline__ bool resolve_row_exact(RSmem& sm, const float* __restrict__ x, int V,
                                                float m, int k, float p, float mu, uint32_t kt,
@@ -1052,13 +1062,31 @@ struct Plan2 {
 
 constexpr int TCAP = CAP / RT;  // private gather slots per thread, interleaved across threads
 
+// Appends the keys of the elements flagged in gm (bit e: element e of the
+// batch) to this thread's gather slots. Hits are rare, so the warp first ORs
+// its lanes' flags and visits only the element positions that some lane hit
+// (a warp-uniform branch each) instead of predicating all eight.
+template <typename KF>
+__device__ __forceinline__ void append_hits(unsigned gm, unsigned long long* tbuf, int& tfill,
+                                            KF&& key_of) {
+  const unsigned wm = __reduce_or_sync(0xffffffffu, gm);
+  if (wm == 0u) return;
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if ((wm >> e) & 1u) {
+      if ((gm >> e) & 1u) {
+        if (tfill < TCAP) tbuf[tfill * RT] = key_of(e);
+        ++tfill;
+      }
+    }
+}
+
 // One pass over the row: exact float64 masses accumulated in registers, and
-// the elements of up to two bucket ranges gathered into per-warp slices of
-// sm.cand with a warp-uniform fill level (ballot + popc: no shared counters).
-// The mass polynomial of E consecutive elements is evaluated as independent
-// chains and summed into split accumulators, so float64 latency is covered.
-// Every lane of a warp runs every batch (invalid slots masked), so the warp
-// votes always see the full warp.
+// the elements of up to two bucket ranges gathered into per-thread slots of
+// sm.cand. The mass polynomial of E consecutive elements is evaluated as
+// independent chains and summed into split accumulators, so float64 latency
+// is covered. Every lane of a warp runs every batch (invalid slots masked), so
+// the warp votes always see the full warp.
 template <bool VEC, bool NEED_Z, bool COUNTS>
 __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, int V, float m,
                                         const Plan2 pl, Pass2& P) {
@@ -1165,16 +1193,9 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
       const bool g = ok(e) && (b - g1s <= g1n || b - g2s <= g2n);
       gm |= g ? 1u << e : 0u;
     }
-    // hits are rare: a vote skips batches without any; each thread appends to
-    // its own slots (no coordination between lanes)
-    if (__any_sync(0xffffffffu, gm != 0u)) {
-#pragma unroll
-      for (int e = 0; e < E; ++e)
-        if ((gm >> e) & 1u) {
-          if (tfill < TCAP) tbuf[tfill * RT] = ckey(sv[e], idx(e));
-          ++tfill;
-        }
-    }
+    // each thread appends its hits to its own slots (no coordination between
+    // lanes)
+    append_hits(gm, tbuf, tfill, [&](int e) { return ckey(sv[e], idx(e)); });
   };
 
   const int tid = (int)threadIdx.x;
@@ -1217,9 +1238,73 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
   P.overflow = __syncthreads_or(tfill > TCAP) != 0;
 }
 
+// A pass that only gathers: the elements of up to two bucket ranges, tested
+// by value against the ranges widened by a bucket on each side (a superset:
+// the readers select the exact buckets), so no bucket index is formed.
+template <bool VEC>
+__device__ __noinline__ void gather_pass(RSmem& sm, const float* __restrict__ x, int V, float m,
+                                         const Plan2 pl, Pass2& P) {
+  constexpr int E = 8;
+  auto widen = [&](int lo, int hi, float& vlo, float& vhi) {
+    if (lo > hi) {
+      vlo = INFINITY;
+      vhi = -INFINITY;
+      return;
+    }
+    vlo = hi >= NB - 1 ? -INFINITY : m - (float)(hi + 2) * (1.0f / BIN_SCALE);
+    vhi = lo <= 0 ? INFINITY : m - (float)(lo - 1) * (1.0f / BIN_SCALE);
+  };
+  float l1, h1, l2, h2;
+  widen(pl.g_lo, pl.g_hi, l1, h1);
+  widen(pl.g2_lo, pl.g2_hi, l2, h2);
+  const int tid = (int)threadIdx.x;
+  unsigned long long* tbuf = sm.cand + tid;
+  int tfill = 0;
+  auto batch = [&](auto full, const float (&sv)[E], int a0, int na, int b0, int nb) {
+    auto idx = [&](int e) { return e < 4 ? a0 + e : b0 + (e - 4); };
+    auto ok = [&](int e) { return decltype(full)::value || (e < 4 ? e < na : e - 4 < nb); };
+    unsigned gm = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float s = sv[e];
+      const bool g = ok(e) && ((s >= l1 && s <= h1) || (s >= l2 && s <= h2));
+      gm |= g ? 1u << e : 0u;
+    }
+    append_hits(gm, tbuf, tfill, [&](int e) { return ckey(sv[e], idx(e)); });
+  };
+  int tail0 = 0;
+  if (VEC) {
+    const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
+    const int V4 = V >> 2;
+    stream_chunks(sm, x4, V4, n_chunks(V4), [](int j) { return j; }, l2_policy_drop(),
+                  [&](auto full, const float4& a4, int ia, const float4& b4, int ib, bool va,
+                      bool vb) {
+                    const float sv[E] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+                    batch(full, sv, 4 * ia, va ? 4 : 0, 4 * ib, vb ? 4 : 0);
+                  });
+    tail0 = 4 * V4;
+  }
+  for (int i0 = tail0; i0 < V; i0 += RT) {
+    const int i = i0 + tid;
+    const bool in = i < V;
+    const float s = in ? ld_stream(x + i) : 0.f;
+    const float sv[E] = {s, s, s, s, s, s, s, s};
+    batch(std::false_type{}, sv, i, in ? 1 : 0, i, 0);
+  }
+  sm.tcount[tid] = tfill;
+  P.z = P.a_p = P.a_mu = P.zx = P.a_px = P.a_mux = 0.0;
+  P.c_p = P.c_mu = 0;
+  P.k_last = ~0ull;
+  P.overflow = __syncthreads_or(tfill > TCAP) != 0;
+}
+
 template <bool VEC>
 __device__ void pass2(RSmem& sm, const float* __restrict__ x, int V, float m, bool need_z,
                       const Plan2& pl, Pass2& P, bool counts = false) {
+  if (!need_z && !counts && pl.b_mu < 0 && !pl.need_last) {  // nothing weighed or counted
+    gather_pass<VEC>(sm, x, V, m, pl, P);
+    return;
+  }
   if (counts) {
     if (need_z)
       pass2_impl<VEC, true, true>(sm, x, V, m, pl, P);
@@ -1253,7 +1338,7 @@ static_assert(MU_SLOTS >= 16, "a thread stages up to 7 + 8 values");
 
 // Level-0 bucket of s as an int and as a float (the same floor as bin0).
 __device__ __forceinline__ int bin0_both(float s, float m, float& bf) {
-  const float f = fminf(fmaxf((m - s) * BIN_SCALE, 0.0f), (float)(NB - 1));
+  const float f = fminf(fmaxf(fmaf(s, -BIN_SCALE, m * BIN_SCALE), 0.0f), (float)(NB - 1));
   const float fl = __fadd_rd(f, 8388608.0f);
   bf = fl - 8388608.0f;
   return __float_as_int(fl) - 0x4B000000;
@@ -1316,14 +1401,7 @@ __device__ __noinline__ void mu_pass(RSmem& sm, const float* __restrict__ x, int
         if (j + E < sf) stage[j * RT] = stage[(j + E) * RT];
       sf -= n;
     }
-    if (__any_sync(0xffffffffu, gm != 0u)) {
-#pragma unroll
-      for (int e = 0; e < E; ++e)
-        if ((gm >> e) & 1u) {
-          if (tfill < TCAP) tbuf[tfill * RT] = ckey(sv[e], idx(e));
-          ++tfill;
-        }
-    }
+    append_hits(gm, tbuf, tfill, [&](int e) { return ckey(sv[e], idx(e)); });
   };
 
   int tail0 = 0;
@@ -1358,6 +1436,112 @@ __device__ __noinline__ void mu_pass(RSmem& sm, const float* __restrict__ x, int
   out.qx = sums[1];
   out.rest_lower = sums[2];
   out.cnt = (long long)sums[3];
+  out.overflow = __syncthreads_or(tfill > TCAP) != 0;
+}
+
+// ---------------------------------------------------------------- fp32-mass passes
+// Identity rows and rows whose min-p prefix decides need no comparison of
+// masses to find their support (min-p compares values), only the support's
+// mass for LSE_S and, with top-p on, a certificate that the top-p crossing
+// comes after the min-p prefix. Without the entropy output (and outside the
+// sampler, whose inverse CDF compares masses) they are weighed in fp32:
+// q = ex2((s - m) log2 e), d = s - m and the product each rounded once, eight
+// terms summed in fp32 per batch and the batch sums added in float64.
+//
+// Error bound (u = 2^-24): the exponent is off by at most 3u |y| (three
+// roundings), so a term's relative error is at most 3u |d| plus ex2.approx's
+// own (a few ulp). Over a set of n terms containing the row max (d = 0,
+// q = 1, so Z >= 1), sum q |d| = Z (H - ln Z) <= Z ln n with H the set's
+// Shannon entropy; the relative error of the sum is therefore at most
+// 3u ln(2^31) + 7u (the batch sums) = 4.3e-6 plus ex2.approx's. MASS_EPS =
+// 2e-5 covers it with room for an ex2 error of 100 ulp.
+constexpr double MASS_EPS = 2e-5;
+
+struct FastPass {
+  double kept, rest;           // masses of the kept elements and of the others
+  long long cnt;               // kept elements
+  unsigned long long k_last;   // identity rows: the last element of the order
+  bool overflow;               // the gather slots overflowed (min-p rows)
+};
+
+// MODE 0 (identity): every element is kept; each thread tracks its smallest
+// value and, among equal ones, its largest id (its elements come in increasing
+// id order, so "<=" takes the later one), which gives the last element of the
+// (s desc, id asc) order. MODE 1 (min-p): an element is kept iff s >= thr;
+// kept elements with s <= hv are gathered (hv bounds the buckets that hold
+// the last kept element, with a bucket of slack).
+template <bool VEC, int MODE>
+__device__ __noinline__ void fast_pass(RSmem& sm, const float* __restrict__ x, int V, float m,
+                                       float thr, float hv, FastPass& out) {
+  constexpr int E = 8;
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int tid = (int)threadIdx.x;
+  unsigned long long* tbuf = sm.cand + tid;
+  int tfill = 0, cnt = 0;
+  double kd = 0.0, rd = 0.0;
+  float vmin = INFINITY;
+  int imax = -1;
+
+  auto batch = [&](auto full, const float (&sv)[E], int a0, int na, int b0, int nb) {
+    auto idx = [&](int e) { return e < 4 ? a0 + e : b0 + (e - 4); };
+    auto ok = [&](int e) { return decltype(full)::value || (e < 4 ? e < na : e - 4 < nb); };
+    float bk = 0.0f, br = 0.0f;
+    unsigned gm = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float q = ex2_approx((sv[e] - m) * kLog2e);
+      if (MODE == 0) {
+        if (ok(e)) {
+          bk += q;
+          if (sv[e] <= vmin) {
+            vmin = sv[e];
+            imax = idx(e);
+          }
+        }
+      } else {
+        const bool kept = ok(e) && sv[e] >= thr;
+        if (kept) {
+          bk += q;
+          ++cnt;
+        } else if (ok(e)) {
+          br += q;
+        }
+        gm |= (kept && sv[e] <= hv) ? 1u << e : 0u;
+      }
+    }
+    kd += (double)bk;
+    if (MODE == 1) {
+      rd += (double)br;
+      append_hits(gm, tbuf, tfill, [&](int e) { return ckey(sv[e], idx(e)); });
+    }
+  };
+
+  int tail0 = 0;
+  if (VEC) {
+    const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
+    const int V4 = V >> 2;
+    stream_chunks(sm, x4, V4, n_chunks(V4), [](int j) { return j; }, l2_policy_drop(),
+                  [&](auto full, const float4& a4, int ia, const float4& b4, int ib, bool va,
+                      bool vb) {
+                    const float sv[E] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+                    batch(full, sv, 4 * ia, va ? 4 : 0, 4 * ib, vb ? 4 : 0);
+                  });
+    tail0 = 4 * V4;
+  }
+  for (int i0 = tail0; i0 < V; i0 += RT) {
+    const int i = i0 + tid;
+    const bool in = i < V;
+    const float s = in ? ld_stream(x + i) : 0.f;
+    const float sv[E] = {s, s, s, s, s, s, s, s};
+    batch(std::false_type{}, sv, i, in ? 1 : 0, i, 0);
+  }
+  sm.tcount[tid] = tfill;
+  double sums[3] = {kd, rd, (double)cnt};
+  block_sum_multi<3>(sums, sm);
+  out.kept = sums[0];
+  out.rest = sums[1];
+  out.cnt = (long long)sums[2];
+  out.k_last = MODE == 0 ? block_ext_u<false>(imax >= 0 ? ckey(vmin, imax) : ~0ull, sm) : ~0ull;
   out.overflow = __syncthreads_or(tfill > TCAP) != 0;
 }
 
@@ -1627,7 +1811,7 @@ __device__ __noinline__ bool resolve_large_k(RSmem& sm, const float* __restrict_
 template <bool VEC>
 __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict__ x, int V, float m,
                                               int k, float p, float mu, uint32_t kt, bool sampled,
-                                              bool ent, Cut& best) {
+                                              bool ent, bool f32m, Cut& best) {
   const bool k_on = k >= 1 && k < V, p_on = p < 1.0f, mu_on = mu > 0.0f;
   Plan2 pl;
   pl.need_last = 0;
@@ -1641,6 +1825,12 @@ __device__ __noinline__ bool resolve_row_fast(RSmem& sm, const float* __restrict
   Pass2 P;
 
   if (!k_on && !p_on && !mu_on) {  // identity: total mass and the last element only
+    if (f32m) {
+      FastPass fp;
+      fast_pass<VEC, 0>(sm, x, V, m, 0.0f, 0.0f, fp);
+      best = Cut{fp.k_last, (long long)V, fp.kept, 0.0};
+      return true;
+    }
     pl.need_last = 1;
     pass2<VEC>(sm, x, V, m, true, pl, P);
     best = Cut{P.k_last, (long long)V, P.z, P.zx};
@@ -1956,7 +2146,7 @@ __device__ __noinline__ void gathered_kept(RSmem& sm, float m, int lo, int hi, u
 template <bool VEC>
 __device__ __noinline__ bool resolve_row_planned(RSmem& sm, const float* __restrict__ x, int V,
                                                  float m, int k, float p, float mu, uint32_t kt,
-                                                 bool ent, bool& sampled, Cut& best) {
+                                                 bool ent, bool f32m, bool& sampled, Cut& best) {
   const bool k_on = k >= 1 && k < V, p_on = p < 1.0f, mu_on = mu > 0.0f;
   sampled = false;
   if (!k_on && !p_on && !mu_on) return false;  // identity rows: the fast path's single pass
@@ -2015,6 +2205,28 @@ __device__ __noinline__ bool resolve_row_planned(RSmem& sm, const float* __restr
   const int bm = bin0(key32_value(kt), m);
   const int g2lo = sampled_before(sm, bm);
   if (p_on && estimated_mass_before(sm, bm + 1) > (double)p - 0.05) return false;
+  if (f32m) {
+    // kept iff s >= thr; the last kept element lies in buckets [g2lo, bm],
+    // so the kept elements with s <= hv (one bucket of slack) are gathered
+    const int glo = g2lo > 0 ? g2lo - 1 : 0;
+    const double est = scale * (double)count_range(sm, glo, bm + 1);
+    if (count_upper(est, scale) > 0.75 * CAP) return false;
+    const float hv = m - (float)(g2lo - 1) * (1.0f / BIN_SCALE);
+    FastPass fp;
+    fast_pass<VEC, 1>(sm, x, V, m, key32_value(kt), hv, fp);
+    if (fp.overflow) return false;
+    const int ng = pack_gathered(sm);
+    if (ng == 0 || ng >= SCAP) return false;
+    const unsigned long long* g = packed(sm);
+    unsigned long long kmn = ~0ull;
+    for (int i = threadIdx.x; i < ng; i += RT) kmn = g[i] < kmn ? g[i] : kmn;
+    const unsigned long long kmin = block_ext_u<false>(kmn, sm);
+    // certificate against the bounds of the fp32 masses
+    if (p_on && !(fp.kept * (1.0 + MASS_EPS) < (double)p * (fp.kept + fp.rest) * (1.0 - MASS_EPS)))
+      return false;
+    best = Cut{kmin, fp.cnt, fp.kept, 0.0};
+    return true;
+  }
   const double est = scale * (double)count_range(sm, g2lo, bm + 1);
   if (count_upper(est, scale) > 0.75 * CAP) return false;  // keep the warp slices far from full
   MuPass mp;
@@ -2139,10 +2351,12 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
     int path = (k_on || p_on || mu_on) ? kPathPlanned : kPathIdentity;
     bool sampled = false;
     const bool ent = a.entropy != nullptr;
-    bool ok = resolve_row_planned<VEC>(sm, x, V, m, k, p, mu, kt, ent, sampled, best);
+    // fp32 masses where no mass comparison decides the output
+    const bool f32m = !ent && a.mode != kModeSample;
+    bool ok = resolve_row_planned<VEC>(sm, x, V, m, k, p, mu, kt, ent, f32m, sampled, best);
     if (!ok) {
       if (path == kPathPlanned) path = kPathFast;
-      ok = resolve_row_fast<VEC>(sm, x, V, m, k, p, mu, kt, sampled, ent, best);
+      ok = resolve_row_fast<VEC>(sm, x, V, m, k, p, mu, kt, sampled, ent, f32m, best);
     }
     if (!ok) {
       path = kPathExact;

@@ -168,3 +168,24 @@ class OraclePool:
 
     def logit_grad(self, s, rows, g):
         return np.concatenate(self.map_rows("logit_grad", s, rows, per_row_extra=(g,)))
+
+
+F32_MASS_LP_ATOL = 3e-5  # logprob of the fp32-mass forward against the float64-mass one
+
+
+def assert_same_decisions(lp_a, saved_a, lp_b, saved_b):
+    """Two forwards of the same rows, one with the entropy output (float64
+    masses) and one without (fp32 masses where no mass comparison decides the
+    support): identical support decisions, logprobs within the fp32 mass
+    bound (relative 2e-5 on the support mass, so 2e-5 on its log, plus the
+    fp32 rounding of LSE_S)."""
+    for key in ("support_size", "cut_id", "cut_logit", "flags"):
+        a, b = saved_a[key], saved_b[key]
+        same = (a == b) | (torch.isnan(a) & torch.isnan(b)) if a.is_floating_point() else a == b
+        assert bool(same.all()), key
+    fin = torch.isfinite(lp_a)
+    assert torch.equal(fin, torch.isfinite(lp_b))
+    assert torch.equal(torch.isnan(lp_a), torch.isnan(lp_b))
+    assert torch.equal(lp_a[~fin & ~torch.isnan(lp_a)], lp_b[~fin & ~torch.isnan(lp_b)])
+    if bool(fin.any()):
+        assert (lp_a[fin] - lp_b[fin]).abs().max().item() < F32_MASS_LP_ATOL

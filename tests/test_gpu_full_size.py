@@ -10,6 +10,9 @@ Checks, each able to fail on any sampled row:
   2. logprob and target membership on every row: against the oracle's, or,
      where the support size legitimately differs, against the oracle's
      logprob on the GPU's support (within 2e-3);
+  2b. the forward without the entropy output (the benchmark's, with fp32
+     masses where no mass comparison decides the support): the same support
+     decisions on every row and its logprob within 3e-5 of the other's;
   3. the forward's cuts (support size, cut id, cut logit) bit-exact against
      the oracle's support program run on the GPU's own fp32 logits of the
      same rows (same fp32 values, every decision in float64 on both sides);
@@ -30,8 +33,8 @@ import torch
 
 import oracle
 import workloads
-from helpers import (GAP_EPS, GRAD_RTOL, OraclePool, bf16_tensor, compare_logprob, f32_values,
-                     grad_rows, rel_fro)
+from helpers import (GAP_EPS, GRAD_RTOL, OraclePool, assert_same_decisions, bf16_tensor,
+                     compare_logprob, f32_values, grad_rows, rel_fro)
 
 pytestmark = pytest.mark.gpu
 
@@ -79,6 +82,15 @@ def test_full_size_workload(cuda_lib, pool, index):
     lp, saved, _ = sts.sts_forward(Hd, Wd, y_t, tau, k, p, mu, check=True, entropy=True)
     lp_sel = lp.cpu().numpy()[sel]
     sv = {n: v.cpu().numpy()[sel] for n, v in saved.items()}
+    # the benchmark's forward (no entropy output: fp32 masses where no mass
+    # comparison decides the support): the same decisions on every row, its
+    # logprob within the fp32 mass bound of the float64-mass one, and within
+    # the oracle tolerance on the sampled rows
+    lp32, saved32, _ = sts.sts_forward(Hd, Wd, y_t, tau, k, p, mu, check=True)
+    assert_same_decisions(lp, saved, lp32, saved32)
+    bad32, _, err32 = compare_logprob(lp32.cpu().numpy()[sel], sv["support_size"], s_sel, rows_sel,
+                                      ref, flagged)
+    assert bad32 == 0, (bad32, err32)
 
     # 1 and 2: against the float64 oracle
     bad, ndiff, max_err = compare_logprob(lp_sel, sv["support_size"], s_sel, rows_sel, ref, flagged)

@@ -12,8 +12,8 @@ import torch
 import oracle
 import workloads
 from sampling_transform_lm_b200.dp import SliceAllReduce
-from helpers import (GRAD_RTOL, bf16_tensor, compare_logprob, f32_values, grad_rows,
-                     near_gap_rows, rel_fro, row_tensors, small_case)
+from helpers import (GRAD_RTOL, assert_same_decisions, bf16_tensor, compare_logprob, f32_values,
+                     grad_rows, near_gap_rows, rel_fro, row_tensors, small_case)
 
 pytestmark = pytest.mark.gpu
 
@@ -25,6 +25,10 @@ def _run(sts, H, W, rows, grad=None, row_chunk=0, vocab_chunk=0):
     y, tau, k, p, mu = row_tensors(rows)
     lp, saved, ws = sts.sts_forward(Hd, Wd, y, tau, k, p, mu, row_chunk=row_chunk, entropy=True)
     status, bad = sts.sts_get_status(ws)
+    # the same rows without the entropy output take fp32 masses where no mass
+    # comparison decides: identical decisions, logprob within the mass bound
+    lp2, saved2, _ = sts.sts_forward(Hd, Wd, y, tau, k, p, mu, row_chunk=row_chunk)
+    assert_same_decisions(lp, saved, lp2, saved2)
     out = {"logprob": lp.cpu().numpy(), "saved": {k_: v.cpu().numpy() for k_, v in saved.items()},
            "status": status, "bad_row": bad}
     if grad is not None:
