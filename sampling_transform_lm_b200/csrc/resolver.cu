@@ -23,7 +23,7 @@
 // metadata and the projection epilogue's per-tile maxima, which give the
 // unfiltered max m, are loaded one row ahead). Rows with a 16-byte aligned
 // start stream through a shared-memory ring filled by bulk copies (one thread
-// keeps four 16 KB chunks in flight), so no pass holds its loads in registers.
+// keeps two 32 KB chunks in flight), so no pass holds its loads in registers.
 //
 //   buckets      floor((m - s) * 128), clamped to 4095: monotone in s, so
 //                every bucket is a contiguous run of the order.
@@ -95,8 +95,9 @@ constexpr float BIN_SCALE = 128.f;  // level-0 buckets per logit unit
 constexpr int MAX_LEVELS = 8;
 constexpr int UNROLL = 4;           // float4 loads in flight per thread
 constexpr int SAMPLE_EVERY = 8;     // the planning sample reads one chunk in 8
-constexpr int CH_F4 = 2 * RT;       // float4s of a streamed chunk (two per thread)
-constexpr int NSTAGE = 4;           // chunks in flight in the shared-memory ring
+constexpr int CPT = 4;              // float4s per thread in a streamed chunk (even)
+constexpr int CH_F4 = CPT * RT;     // float4s of a streamed chunk (32 KB)
+constexpr int NSTAGE = 2;           // chunks in flight in the shared-memory ring
 
 // exp(-b / 128) for every bucket b.
 struct ExpTab {
@@ -288,13 +289,15 @@ __device__ __forceinline__ void for_each(const float* __restrict__ x, int V, F&&
 // (chunk c = float4s [c CH_F4, min(V4, (c + 1) CH_F4))) that bulk copies put
 // into the shared-memory ring. Up to NSTAGE copies are in flight, so a pass's
 // HBM latency is covered without holding loads in registers; every thread
-// takes the float4s at offsets t and t + RT of each chunk, and the warp that
-// finishes a chunk last copies the chunk NSTAGE ahead into its slot.
+// takes the float4s at offsets t, t + RT, ..., t + (CPT - 1) RT of each chunk,
+// two per batch, and the warp that finishes a chunk last copies the chunk
+// NSTAGE ahead into its slot. Large chunks (32 KB) amortise each chunk's wait
+// and hand-off over 16 elements per thread.
 //
 // stream_chunks streams chunks chunk_of(0), ..., chunk_of(n - 1) and calls
-// f(full, a, ia, b, ib, va, vb) for each: a and b the thread's two float4s,
-// ia and ib their float4 indices in the row, va and vb whether they lie in the
-// row, and `full` (a type) true at compile time for every chunk but a partial
+// f(full, a, ia, b, ib, va, vb) for each batch: a and b two of the thread's
+// float4s, ia and ib their float4 indices in the row, va and vb whether they
+// lie in the row, and `full` (a type) true at compile time for every chunk but a partial
 // last one. sm.ring_q[t] counts the chunks the CTA has consumed so far (the
 // same on every thread); it fixes the parity of every ring barrier. Returns
 // false when a bounded wait gave up: sm.abort_flag is then raised,
@@ -333,12 +336,18 @@ __device__ __forceinline__ bool stream_chunks(RSmem& sm, const float4* __restric
     }
     const int f0 = chunk_of(j) * CH_F4;
     const int cnt = min(CH_F4, V4 - f0);
-    const float4 a = sm.ring[s][tid];
-    const float4 b = sm.ring[s][tid + RT];
-    if (cnt == CH_F4)
-      f(std::true_type{}, a, f0 + tid, b, f0 + tid + RT, true, true);
-    else
-      f(std::false_type{}, a, f0 + tid, b, f0 + tid + RT, tid < cnt, tid + RT < cnt);
+    // the thread's float4s of the chunk, two per batch, in increasing index
+    // (one copy of the batch code: the heavy passes keep their registers)
+#pragma unroll 1
+    for (int h = 0; h < CPT; h += 2) {
+      const int ia = tid + h * RT, ib = ia + RT;
+      const float4 a = sm.ring[s][ia];
+      const float4 b = sm.ring[s][ib];
+      if (cnt == CH_F4)
+        f(std::true_type{}, a, f0 + ia, b, f0 + ib, true, true);
+      else
+        f(std::false_type{}, a, f0 + ia, b, f0 + ib, ia < cnt, ib < cnt);
+    }
     __syncwarp();
     // the warp that finishes a chunk last refills its slot: no warp waits for
     // another one to release a slot
@@ -1062,6 +1071,10 @@ struct Plan2 {
 
 constexpr int TCAP = CAP / RT;  // private gather slots per thread, interleaved across threads
 
+// Per-element tests in the streaming passes combine their comparisons with
+// bitwise & and | rather than && and ||: the short-circuit forms compile to
+// branches, which halved a pass's throughput in a streaming microbenchmark.
+//
 // Appends the keys of the elements flagged in gm (bit e: element e of the
 // batch) to this thread's gather slots. Hits are rare, so the warp first ORs
 // its lanes' flags and visits only the element positions that some lane hit
@@ -1168,15 +1181,15 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
             zx += qx;
             if (bb[e] < w_lo) apx += qx;
           }
-          if (need_mu && bb[e] < b_mu) amux += qx;
+          if (need_mu & (bb[e] < b_mu)) amux += qx;
         }
       }
     }
     if (COUNTS) {
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        if (ok(e) && bb[e] < w_lo) ++cp;
-        if (ok(e) && bb[e] < b_mu) ++cmu;
+        cp += (int)(ok(e) & (bb[e] < w_lo));
+        cmu += (int)(ok(e) & (bb[e] < b_mu));
       }
     }
     if (need_last) {
@@ -1190,7 +1203,7 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const unsigned b = (unsigned)bb[e];
-      const bool g = ok(e) && (b - g1s <= g1n || b - g2s <= g2n);
+      const bool g = ok(e) & ((b - g1s <= g1n) | (b - g2s <= g2n));
       gm |= g ? 1u << e : 0u;
     }
     // each thread appends its hits to its own slots (no coordination between
@@ -1201,8 +1214,8 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
   const int tid = (int)threadIdx.x;
   int tail0 = 0;  // first token handled one per thread
   if (VEC) {
-    // the row streams through the ring; a batch is the thread's two float4s
-    // of a chunk (the loads read evict-first: this is the row's last pass)
+    // the row streams through the ring; a batch is two of the thread's
+    // float4s of a chunk (the loads read evict-first: this is the row's last pass)
     const float4* __restrict__ x4 = reinterpret_cast<const float4*>(x);
     const int V4 = V >> 2;
     stream_chunks(sm, x4, V4, n_chunks(V4), [](int j) { return j; }, l2_policy_drop(),
@@ -1267,7 +1280,7 @@ __device__ __noinline__ void gather_pass(RSmem& sm, const float* __restrict__ x,
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const float s = sv[e];
-      const bool g = ok(e) && ((s >= l1 && s <= h1) || (s >= l2 && s <= h2));
+      const bool g = ok(e) & (((s >= l1) & (s <= h1)) | ((s >= l2) & (s <= h2)));
       gm |= g ? 1u << e : 0u;
     }
     append_hits(gm, tbuf, tfill, [&](int e) { return ckey(sv[e], idx(e)); });
@@ -1385,12 +1398,12 @@ __device__ __noinline__ void mu_pass(RSmem& sm, const float* __restrict__ x, int
       float bf;
       const int b = bin0_both(sv[e], m, bf);
       const bool v = ok(e);
-      if (v && b < g_lo) {
+      if (v & (b < g_lo)) {
         stage[sf * RT] = sv[e];
         ++sf;
       }
-      gm |= (v && (unsigned)b - gs <= gn) ? 1u << e : 0u;
-      if (v && b > g_hi) rest += ex2_approx(-(bf + 1.0f) * kL);
+      gm |= (unsigned)(v & ((unsigned)b - gs <= gn)) << e;
+      if (v & (b > g_hi)) rest += ex2_approx(-(bf + 1.0f) * kL);
     }
     if (__any_sync(0xffffffffu, sf >= E)) {  // weigh eight, keep the rest staged
       const int n = min(sf, E);
@@ -1499,14 +1512,14 @@ __device__ __noinline__ void fast_pass(RSmem& sm, const float* __restrict__ x, i
           }
         }
       } else {
-        const bool kept = ok(e) && sv[e] >= thr;
+        const bool kept = ok(e) & (sv[e] >= thr);
         if (kept) {
           bk += q;
           ++cnt;
         } else if (ok(e)) {
           br += q;
         }
-        gm |= (kept && sv[e] <= hv) ? 1u << e : 0u;
+        gm |= (unsigned)(kept & (sv[e] <= hv)) << e;
       }
     }
     kd += (double)bk;
