@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define STS_ABI_VERSION 2
+#define STS_ABI_VERSION 3
 
 /* cudaStream_t without pulling in the CUDA headers (same opaque type). */
 typedef struct CUstream_st* sts_stream_t;
@@ -212,6 +212,48 @@ sts_status sts_backward_shard(const sts_shape* shape, const void* H_bf16, const 
                               const float* grad_logprob, float* dH_partial, float* dW_shard,
                               int accumulate_dW, int64_t vocab_offset, void* ws, size_t ws_bytes,
                               sts_stream_t stream);
+
+/* The statistics merge: the same support program with per-row statistics
+ * crossing the ranks instead of logits. Every rank runs the four stages on
+ * its own shard S [T, ld] (fp32 scaled logits of vocabulary rows
+ * [vocab_offset, vocab_offset + Vl) of V), and the caller combines each
+ * stage's outputs over the ranks before the next stage:
+ *   1. sts_tp_row_max -> row_max [T]; combine by max: m.
+ *   2. sts_tp_count(m) -> counts [T][buckets] int32 of floor((m - s) 128)
+ *      clamped to buckets - 1; combine by sum.
+ *   3. sts_tp_exact(m, merged counts) -> plan [T][plan_fields] (identical on
+ *      every rank), sums [T][sum_fields] float64 (combine by sum), keys
+ *      [T][key_fields] int64 (combine by min), ylogit [T][2] (combine by sum),
+ *      cand [T][cap] uint64 composite keys and ncand [T] (all-gather both, in
+ *      rank order: [world][T][cap] and [world][T]).
+ *   4. sts_tp_finish -> logprob and the saved scalars of sts_forward, for
+ *      every row where need_gather[r] == 0; need_gather[r] == 1 (the same on
+ *      every rank) marks a row whose gathered buckets did not hold its top-p
+ *      crossing, or held more keys than one sort (sort_cap) or than a rank's
+ *      cap: resolve it from gathered full rows instead
+ *      (sts_gather_vocab_shards + sts_resolve_logits). Rows are
+ *      validated here (invalid rows: NaN, flag STS_ROW_INVALID, status in
+ *      ws, which holds at least the 256-byte status header).
+ * Masses are float64 (no fp32-mass shortcut); entropy is not formed.
+ * sts_tp_constants reports buckets, plan_fields, sum_fields, key_fields and
+ * sort_cap. All pointers are device memory except the constants' outputs;
+ * calls are asynchronous on `stream` and allocate nothing. STS_ERR_SHAPE for
+ * inconsistent sizes (ld < Vl, vocab_offset + Vl > V, cap < 1). */
+sts_status sts_tp_constants(int64_t* buckets, int64_t* plan_fields, int64_t* sum_fields,
+                            int64_t* key_fields, int64_t* sort_cap);
+sts_status sts_tp_row_max(const float* S, int64_t T, int64_t Vl, int64_t ld, float* row_max,
+                          sts_stream_t stream);
+sts_status sts_tp_count(const float* S, int64_t T, int64_t Vl, int64_t ld, const float* m,
+                        int32_t* counts, sts_stream_t stream);
+sts_status sts_tp_exact(const float* S, int64_t T, int64_t Vl, int64_t ld, int64_t vocab_offset,
+                        int64_t V, const sts_rows* rows, const float* m, const int32_t* counts,
+                        int32_t* plan, double* sums, int64_t* keys, float* ylogit, uint64_t* cand,
+                        int32_t* ncand, int64_t cap, sts_stream_t stream);
+sts_status sts_tp_finish(int64_t T, int64_t V, int64_t world, const sts_rows* rows, const float* m,
+                         const int32_t* plan, const double* sums, const int64_t* keys,
+                         const float* ylogit, const uint64_t* cand, const int32_t* ncand,
+                         int64_t cap, float* logprob, const sts_saved* saved,
+                         int32_t* need_gather, void* ws, size_t ws_bytes, sts_stream_t stream);
 
 /* Draw one token per row from the filtered distribution: the inverse CDF of
  * the support walked in (s desc, id asc) order, taking the first kept token

@@ -35,6 +35,11 @@ __all__ = [
     "sts_backward_shard",
     "sts_resolve_logits",
     "sts_gather_vocab_shards",
+    "sts_tp_constants",
+    "sts_tp_row_max",
+    "sts_tp_count",
+    "sts_tp_exact",
+    "sts_tp_finish",
     "VocabParallel",
     "SliceAllReduce",
     "sts_sample",
@@ -92,6 +97,11 @@ EXPORTED_SYMBOLS = (
     "sts_backward_shard",
     "sts_resolve_logits",
     "sts_gather_vocab_shards",
+    "sts_tp_constants",
+    "sts_tp_row_max",
+    "sts_tp_count",
+    "sts_tp_exact",
+    "sts_tp_finish",
 )
 
 
@@ -162,6 +172,19 @@ def load():
     lib.sts_resolve_logits.restype = ctypes.c_int
     lib.sts_gather_vocab_shards.argtypes = [P, I64, I64, I64, P, I64, P]
     lib.sts_gather_vocab_shards.restype = ctypes.c_int
+    PI64 = ctypes.POINTER(ctypes.c_int64)
+    lib.sts_tp_constants.argtypes = [PI64, PI64, PI64, PI64, PI64]
+    lib.sts_tp_constants.restype = ctypes.c_int
+    lib.sts_tp_row_max.argtypes = [P, I64, I64, I64, P, P]
+    lib.sts_tp_row_max.restype = ctypes.c_int
+    lib.sts_tp_count.argtypes = [P, I64, I64, I64, P, P, P]
+    lib.sts_tp_count.restype = ctypes.c_int
+    lib.sts_tp_exact.argtypes = [P, I64, I64, I64, I64, I64, ctypes.POINTER(_Rows), P, P, P, P, P,
+                                 P, P, P, I64, P]
+    lib.sts_tp_exact.restype = ctypes.c_int
+    lib.sts_tp_finish.argtypes = [I64, I64, I64, ctypes.POINTER(_Rows), P, P, P, P, P, P, P, I64, P,
+                                  ctypes.POINTER(_Saved), P, P, S, P]
+    lib.sts_tp_finish.restype = ctypes.c_int
     lib.sts_sample.argtypes = [ctypes.POINTER(_Shape), P, P, ctypes.POINTER(_Rows), P, P, P, S, P]
     lib.sts_sample.restype = ctypes.c_int
     lib.sts_filter_logits.argtypes = [ctypes.POINTER(_Shape), P, ctypes.POINTER(_Rows), P, P, P, P,
@@ -617,6 +640,93 @@ def sts_backward_shard(H, W_shard, target, temperature, top_k, top_p, min_p, sav
     if check:
         sts_get_status(ws, stream, raise_on_error=True)
     return dH, dW
+
+
+def sts_tp_constants():
+    """Sizes of the statistics-merge stages' per-row records."""
+    lib = load()
+    v = [ctypes.c_int64() for _ in range(5)]
+    _check(lib.sts_tp_constants(*(ctypes.byref(x) for x in v)), "sts_tp_constants")
+    return dict(zip(("buckets", "plan_fields", "sum_fields", "key_fields", "sort_cap"),
+                    (int(x.value) for x in v)))
+
+
+def _shard_view(S):
+    _need(S, torch.float32, "S")
+    if S.dim() != 2 or S.stride(1) != 1:
+        raise StsError(STS_ERR_SHAPE, "S must be [T, Vl] with unit column stride")
+    return S.shape[0], S.shape[1], S.stride(0)
+
+
+def sts_tp_row_max(S, *, stream=None):
+    """Stage 1 of the statistics merge: this shard's row maxima [T]."""
+    lib = load()
+    T, Vl, ld = _shard_view(S)
+    out = torch.empty(T, dtype=torch.float32, device=S.device)
+    _check(lib.sts_tp_row_max(_ptr(S), T, Vl, ld, _ptr(out), _stream(stream)), "sts_tp_row_max")
+    return out
+
+
+def sts_tp_count(S, m, *, stream=None):
+    """Stage 2: this shard's bucket counts [T, buckets] against the merged row max m."""
+    lib = load()
+    T, Vl, ld = _shard_view(S)
+    _need(m, torch.float32, "m", (T,))
+    nb = sts_tp_constants()["buckets"]
+    out = torch.empty((T, nb), dtype=torch.int32, device=S.device)
+    _check(lib.sts_tp_count(_ptr(S), T, Vl, ld, _ptr(m), _ptr(out), _stream(stream)),
+           "sts_tp_count")
+    return out
+
+
+def sts_tp_exact(S, vocab_offset, V, target, temperature, top_k, top_p, min_p, m, counts, *,
+                 cap=None, stream=None):
+    """Stage 3: the row plans, float64 sums, smallest keys, target logit and
+    gathered composite keys of this shard (a dict of tensors)."""
+    lib = load()
+    T, Vl, ld = _shard_view(S)
+    c = sts_tp_constants()
+    cap = c["sort_cap"] if cap is None else int(cap)
+    rows = _rows(T, target, temperature, top_k, top_p, min_p)
+    _need(m, torch.float32, "m", (T,))
+    _need(counts, torch.int32, "counts", (T, c["buckets"]))
+    dev = S.device
+    out = {
+        "plan": torch.empty((T, c["plan_fields"]), dtype=torch.int32, device=dev),
+        "sums": torch.empty((T, c["sum_fields"]), dtype=torch.float64, device=dev),
+        "keys": torch.empty((T, c["key_fields"]), dtype=torch.int64, device=dev),
+        "ylogit": torch.empty((T, 2), dtype=torch.float32, device=dev),
+        "cand": torch.empty((T, cap), dtype=torch.int64, device=dev),
+        "ncand": torch.empty(T, dtype=torch.int32, device=dev),
+    }
+    st = lib.sts_tp_exact(_ptr(S), T, Vl, ld, int(vocab_offset), int(V), ctypes.byref(rows), _ptr(m),
+                          _ptr(counts), _ptr(out["plan"]), _ptr(out["sums"]), _ptr(out["keys"]),
+                          _ptr(out["ylogit"]), _ptr(out["cand"]), _ptr(out["ncand"]), cap,
+                          _stream(stream))
+    _check(st, "sts_tp_exact")
+    return out
+
+
+def sts_tp_finish(V, target, temperature, top_k, top_p, min_p, m, plan, sums, keys, ylogit, cand,
+                  ncand, *, ws=None, stream=None):
+    """Stage 4: logprob and saved scalars from the merged stage-3 records
+    (cand [world, T, cap] and ncand [world, T] in rank order). Returns
+    (logprob, saved, need_gather, ws)."""
+    lib = load()
+    world, T, cap = cand.shape
+    rows = _rows(T, target, temperature, top_k, top_p, min_p)
+    dev = m.device
+    _need(ncand, torch.int32, "ncand", (world, T))
+    ws = _workspace(256, dev, ws)
+    logprob = torch.empty(T, dtype=torch.float32, device=dev)
+    saved = _saved_tensors(T, dev)
+    need = torch.empty(T, dtype=torch.int32, device=dev)
+    st = lib.sts_tp_finish(T, int(V), world, ctypes.byref(rows), _ptr(m), _ptr(plan), _ptr(sums),
+                           _ptr(keys), _ptr(ylogit), _ptr(cand), _ptr(ncand), cap, _ptr(logprob),
+                           ctypes.byref(_saved_struct(saved)), _ptr(need), _ptr(ws), ws.numel(),
+                           _stream(stream))
+    _check(st, "sts_tp_finish")
+    return logprob, saved, need, ws
 
 
 def sts_gather_vocab_shards(src, dst, *, stream=None):

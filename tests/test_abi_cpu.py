@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol(lib):
     for name in names:
         assert hasattr(lib, name), name
     assert set(names) == set(sts.EXPORTED_SYMBOLS)
-    assert lib.sts_abi_version() == 2
+    assert lib.sts_abi_version() == 3
 
 
 def test_status_strings(lib):
@@ -176,3 +176,32 @@ def test_policy_grad_host_checks(lib):
     assert lib.sts_policy_grad(4, null, null, null, 0, 0.2, 0.2, float("inf"), null, null) == 2
     assert lib.sts_policy_grad(4, null, null, null, 0, 0.2, 0.2, 1.0, null, null) == 1
     assert lib.sts_policy_grad(0, null, null, null, 1, 0.2, 0.2, 1.0, null, null) == 0
+
+
+def test_statistics_merge_host_checks(lib):
+    """The vocabulary-parallel merge stages: their record sizes, and argument
+    errors returned before any device work (no GPU needed)."""
+    c = sts.sts_tp_constants()
+    assert c == {"buckets": 4096, "plan_fields": 8, "sum_fields": 5, "key_fields": 2,
+                 "sort_cap": 8192}
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(4096)  # never dereferenced: the checks fail first
+    assert lib.sts_tp_row_max(null, 4, 8, 8, fake, None) == 1
+    assert lib.sts_tp_row_max(fake, 4, 8, 7, fake, None) == 2      # ld < Vl
+    assert lib.sts_tp_row_max(fake, 0, 8, 8, fake, None) == 2      # no rows
+    assert lib.sts_tp_count(fake, 4, 8, 8, null, fake, None) == 1
+    assert lib.sts_tp_count(fake, 4, -1, 8, fake, fake, None) == 2
+    rows = _Rows(4, fake, fake, fake, fake, fake)
+    short = _Rows(3, fake, fake, fake, fake, fake)
+    bad_off = [fake, 4, 8, 8, 12, 16, ctypes.byref(rows)] + [fake] * 8
+    assert lib.sts_tp_exact(*bad_off, 4096, None) == 2           # offset + Vl > V
+    assert lib.sts_tp_exact(*([fake, 4, 8, 8, 0, 16, ctypes.byref(short)] + [fake] * 8),
+                            4096, None) == 2                     # metadata length != T
+    assert lib.sts_tp_exact(*([fake, 4, 8, 8, 0, 16, ctypes.byref(rows)] + [fake] * 8),
+                            0, None) == 2                        # cap < 1
+    saved = _Saved(fake, fake, fake, fake, fake, fake)
+    fin = [4, 16, 2, ctypes.byref(rows)] + [fake] * 7 + [4096, fake, ctypes.byref(saved), fake]
+    assert lib.sts_tp_finish(*fin, null, 256, None) == 9          # no workspace
+    assert lib.sts_tp_finish(*fin, fake, 100, None) == 9          # short workspace
+    fin0 = [4, 16, 0, ctypes.byref(rows)] + [fake] * 7 + [4096, fake, ctypes.byref(saved), fake]
+    assert lib.sts_tp_finish(*fin0, fake, 256, None) == 2         # world < 1

@@ -1,9 +1,13 @@
 """Host logic of the vocabulary-parallel path (VocabParallel), on CPU with two
 gloo ranks and per-rank stand-ins for the kernels built from the float64
-oracle: the shards' logits gathered in rank order reproduce the full rows,
-the support program on them gives the unsharded oracle's logprobs, each rank
-keeps its own dW shard and the summed dH equals the unsharded one. The
-library's kernels take the same steps in the GPU tests."""
+oracle, in both forms: the gather (the shards' logits gathered in rank order
+reproduce the full rows) and the statistics merge (the collectives of every
+stage in order -- max, sum, sum / min / sum, two all-gathers -- with stand-in
+stages whose merged keys rebuild the rows, and rows handed to the gather form
+where the merge flags them). Either way the support program gives the
+unsharded oracle's logprobs, each rank keeps its own dW shard and the summed
+dH equals the unsharded one. The library's kernels take the same steps in the
+GPU tests."""
 
 import math
 import multiprocessing as mp
@@ -47,6 +51,67 @@ class OracleOps:
         saved = {"S": S[:, :V].clone(), "size": torch.from_numpy(ref["size"])}
         return torch.from_numpy(ref["logprob"]), saved
 
+    # statistics-merge stand-ins: each rank's "gathered keys" are all of its
+    # keys, so the merged keys rebuild the full rows; every seventh row is
+    # flagged for the gather form
+    def row_max(self, local):
+        return local.max(dim=1).values.clone()
+
+    def count(self, local, m):
+        f = (m[:, None].numpy() - local.numpy()).astype(np.float32) * np.float32(128.0)
+        b = np.clip(np.floor(f), 0, 4095).astype(np.int64)
+        out = np.zeros((local.shape[0], 4096), np.int32)
+        for r in range(local.shape[0]):
+            out[r] = np.bincount(b[r], minlength=4096)
+        return torch.from_numpy(out)
+
+    @staticmethod
+    def _keys(vals, ids):
+        u = vals.astype(np.float32).view(np.uint32).astype(np.uint64)
+        u[u == 0x80000000] = 0
+        k32 = np.where(u & 0x80000000, (~u) & 0xFFFFFFFF, u | 0x80000000)
+        return (k32 << np.uint64(32)) | (np.uint64(0xFFFFFFFF) - ids.astype(np.uint64))
+
+    def sort_cap(self):
+        return 8192
+
+    def exact(self, local, vocab_offset, V, target, temperature, top_k, top_p, min_p, m, counts,
+              cap):
+        rows, vl = local.shape
+        s = local.numpy()
+        K = self._keys(s, np.arange(vocab_offset, vocab_offset + vl)[None, :].repeat(rows, 0))
+        y = target.numpy()
+        mine = (y >= vocab_offset) & (y < vocab_offset + vl)
+        yl = np.zeros((rows, 2), np.float32)
+        yl[mine, 0] = s[mine, y[mine] - vocab_offset]
+        yl[mine, 1] = 1.0
+        flip = np.uint64(1 << 63)
+        return {"plan": torch.zeros((rows, 8), dtype=torch.int32),
+                "sums": torch.from_numpy(np.exp(s.astype(np.float64) - m.numpy()[:, None].astype(
+                    np.float64)).sum(1, keepdims=True).repeat(5, 1)),
+                "keys": torch.from_numpy((K.min(1) ^ flip).view(np.int64)[:, None].repeat(2, 1)),
+                "ylogit": torch.from_numpy(yl),
+                "cand": torch.from_numpy(K.view(np.int64)),
+                "ncand": torch.full((rows,), vl, dtype=torch.int32)}
+
+    def finish(self, V, target, temperature, top_k, top_p, min_p, m, rec, cand, ncand):
+        world, rows, cap = cand.shape
+        assert (ncand.numpy() == cap).all() and world * cap == V
+        K = cand.numpy().view(np.uint64).transpose(1, 0, 2).reshape(rows, V)
+        k32 = (K >> np.uint64(32)).astype(np.uint32)
+        u = np.where(k32 & 0x80000000, k32 & 0x7FFFFFFF, (~k32) & 0xFFFFFFFF).astype(np.uint32)
+        ids = (np.uint64(0xFFFFFFFF) - (K & np.uint64(0xFFFFFFFF))).astype(np.int64)
+        S = np.zeros((rows, V), np.float32)
+        np.put_along_axis(S, ids, u.view(np.float32), axis=1)
+        # the merged records hold each rank's contribution exactly once
+        assert np.allclose(rec["ylogit"].numpy()[:, 1], 1.0)
+        lp, saved = self.resolve(torch.from_numpy(S), V, target, temperature, top_k, top_p,
+                                 min_p, False)
+        need = torch.zeros(rows, dtype=torch.int32)
+        need[::7] = 1
+        lp = torch.where(need.bool(), torch.full_like(lp, float("nan")), lp)
+        return lp, saved, need
+
     def backward_shard(self, H, W_shard, target, temperature, top_k, top_p, min_p, saved, grad,
                        vocab_offset):
         rows = {"target": target.numpy(), "temperature": temperature.numpy(),
@@ -73,7 +138,7 @@ def _case(T=300, d=24, V=512):
     return H, W, dict(meta, target=y), g, s
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, mode="gather"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -81,23 +146,23 @@ def _worker(rank, world, port, q):
         vl = W.shape[0] // world
         Ws = torch.from_numpy(W[rank * vl:(rank + 1) * vl])
         t = {k: torch.from_numpy(np.asarray(v)) for k, v in rows.items()}
-        tp = VocabParallel(ops=OracleOps(), row_chunk=128)
+        tp = VocabParallel(ops=OracleOps(), row_chunk=128, mode=mode)
         lp, saved = tp.forward(torch.from_numpy(H), Ws, t["target"], t["temperature"], t["top_k"],
                                t["top_p"], t["min_p"])
         dH, dW = tp.backward(torch.from_numpy(H), Ws, t["target"], t["temperature"], t["top_k"],
                              t["top_p"], t["min_p"], saved, torch.from_numpy(g))
-        q.put((rank, lp.numpy(), dH.numpy(), dW.numpy()))
+        q.put((rank, lp.numpy(), dH.numpy(), dW.numpy(), tp.gathered_rows))
     finally:
         dist.destroy_process_group()
 
 
-def test_vocab_parallel_two_gloo_ranks():
+def _run_two_ranks(mode):
     with socket.socket() as so:
         so.bind(("127.0.0.1", 0))
         port = so.getsockname()[1]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q, mode)) for r in range(2)]
     for p in procs:
         p.start()
     got = sorted((q.get(timeout=180) for _ in range(2)), key=lambda x: x[0])
@@ -110,7 +175,21 @@ def test_vocab_parallel_two_gloo_ranks():
     dH_ref = dZ @ W.astype(np.float64)
     dW_ref = dZ.T @ H.astype(np.float64)
     vl = W.shape[0] // 2
-    for rank, lp, dH, dW in got:
+    for rank, lp, dH, dW, gathered in got:
         np.testing.assert_array_equal(lp, ref["logprob"])  # same fp32 rows, same program
         np.testing.assert_allclose(dH, dH_ref, rtol=1e-12, atol=1e-12)  # partial sums added
         np.testing.assert_allclose(dW, dW_ref[rank * vl:(rank + 1) * vl], rtol=1e-12, atol=1e-12)
+    return [x[4] for x in got]
+
+
+def test_vocab_parallel_two_gloo_ranks():
+    _run_two_ranks("gather")
+
+
+def test_vocab_parallel_statistics_merge_two_gloo_ranks():
+    """The merge's collectives in order, and the rows it flags (every seventh
+    here) taken from the gather form on both ranks alike."""
+    gathered = _run_two_ranks("merge")
+    T = 300
+    flagged = sum(len(range(0, min(128, T - t0), 7)) for t0 in range(0, T, 128))
+    assert gathered == [flagged, flagged]
