@@ -59,7 +59,7 @@ def _peaks():
 # Which sources each kernel kind's recorded DRAM traffic depends on.
 _TRAFFIC_SOURCES = {
     "gemm": ["gemm_sm100.cuh", "sts_device.cuh", "sts_api.cu"],
-    "resolve": ["resolver.cu", "sts_device.cuh", "sts_internal.h"],
+    "resolve": ["resolver.cu", "support_keys.cuh", "sts_device.cuh", "sts_internal.h"],
 }
 
 
@@ -72,10 +72,12 @@ def source_code_only(text):
     return "\n".join(ln for ln in lines if ln.strip())
 
 
-def recorded_traffic(T, d, V, kernel):
+def recorded_traffic(T, d, V, kernel, launches_per_step=None):
     """DRAM bytes (read + write) per launch of ``kernel`` from the committed
     ncu capture of this workload (profiles/dram_traffic_T*_d*_V*.json), or
-    None when there is none or the kernel's sources changed since."""
+    None when there is none or the kernel's sources changed since. A record
+    kept per row (the resolver's: its traffic grows with the rows a launch
+    resolves) is scaled to the average launch, T / launches_per_step rows."""
     import hashlib
     path = os.path.join(ROOT, "profiles", f"dram_traffic_T{T}_d{d}_V{V}.json")
     if not os.path.exists(path):
@@ -90,6 +92,10 @@ def recorded_traffic(T, d, V, kernel):
     k = rec.get("kernels", {}).get(kernel)
     if k is None or rec.get("sources", {}).get(group) != h.hexdigest()[:16]:
         return None
+    if "dram_bytes_per_row" in k:
+        if not launches_per_step:
+            return None
+        return int(k["dram_bytes_per_row"] * T / launches_per_step)
     return int(k["dram_read_bytes_per_launch"] + k["dram_write_bytes_per_launch"])
 
 
@@ -397,7 +403,7 @@ def kernel_rooflines(kern, steps, T, d, V, peaks):
         achieved = bytes_ * steps / (dom_ms / 1e3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": recorded_traffic(T, d, V, dom), "launches": dom_n,
+                "traffic": recorded_traffic(T, d, V, dom, dom_n / steps), "launches": dom_n,
                 "ms_per_step": round(dom_ms / steps, 3)}
     res_ms, res_n = kern.get("resolve", (0.0, 0))
     roof_res = None
@@ -405,7 +411,8 @@ def kernel_rooflines(kern, steps, T, d, V, peaks):
         gbs = 4.0 * T * V * steps / (res_ms / 1e3) / 1e9
         roof_res = {"kernel": "resolve", "bound": "hbm", "achieved": round(gbs, 1),
                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                    "traffic": recorded_traffic(T, d, V, "resolve"), "launches": res_n,
+                    "traffic": recorded_traffic(T, d, V, "resolve", res_n / steps),
+                    "launches": res_n,
                     "ms_per_step": round(res_ms / steps, 3),
                     "note": "algorithmic bytes: one read of the row's fp32 logits; the resolver "
                             "is bound by instruction issue (float64-exact masses), not bandwidth"}

@@ -114,3 +114,22 @@ def test_reference_arm_json_line():
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_recorded_traffic_per_row_scales_to_the_average_launch(tmp_path, monkeypatch):
+    import hashlib
+    csrc = tmp_path / "sampling_transform_lm_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    h = hashlib.sha256()
+    for name in bench._TRAFFIC_SOURCES["resolve"]:
+        (csrc / name).write_text(f"int {name.split('.')[0]} = 1;  // a comment\n")
+        h.update(bench.source_code_only((csrc / name).read_text()).encode())
+    (tmp_path / "profiles").mkdir()
+    rec = {"sources": {"resolve": h.hexdigest()[:16]},
+           "kernels": {"resolve": {"dram_bytes_per_row": 100.0}}}
+    (tmp_path / "profiles" / "dram_traffic_T8_d4_V16.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic(8, 4, 16, "resolve", 2) == 400  # 8 rows over 2 launches
+    assert bench.recorded_traffic(8, 4, 16, "resolve") is None    # launches unknown
+    (csrc / "resolver.cu").write_text("int changed = 2;\n")
+    assert bench.recorded_traffic(8, 4, 16, "resolve", 2) is None

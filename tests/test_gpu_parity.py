@@ -390,8 +390,8 @@ def test_vocab_shards_reproduce_the_unsharded_path(cuda_lib):
 
 
 def test_vocab_parallel_single_rank_nccl(cuda_lib):
-    """VocabParallel over a one-rank NCCL group (the collectives are the
-    identity): the same logprobs, dH and dW as the unsharded path."""
+    """VocabParallel's gather form over a one-rank NCCL group (the collectives
+    are the identity): the same logprobs, dH and dW as the unsharded path."""
     import datetime
 
     import torch.distributed as dist
@@ -415,7 +415,7 @@ def test_vocab_parallel_single_rank_nccl(cuda_lib):
                             timeout=datetime.timedelta(seconds=60),
                             device_id=torch.device("cuda", torch.cuda.current_device()))
     try:
-        tp = VocabParallel(row_chunk=128)
+        tp = VocabParallel(row_chunk=128, mode="gather")
         lp, saved = tp.forward(Hd, Wd, y, tau, k, p, mu)
         dH, dW = tp.backward(Hd, Wd, y, tau, k, p, mu, saved, g)
         torch.cuda.synchronize()
