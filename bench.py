@@ -267,14 +267,20 @@ def vocab_chunk_label(wl, V):
     return min(vc, (V + 255) // 256 * 256)
 
 
-def workload_config(wl, T, V, world, reduced=False):
+DP_COMM_SMS = 8  # SMs the persistent backward GEMMs leave to the dW exchange (N > 1)
+
+
+def workload_config(wl, T, V, world, reduced=False, exchange=False):
     """The ``config`` object of the JSON line; identical for both arms."""
     return {
         "workload": f"{wl.name}: {wl.desc}" + (
             f" [reduced to T={T}, V={V} for a profiling capture]" if reduced else ""),
         "T_per_gpu": T, "d": wl.d, "V": V, "global_batch": world * T,
         "vocab_chunk": vocab_chunk_label(wl, V),
-        "parallelism": f"dp{world} (one batch per GPU, no collective on the data path)",
+        "parallelism": (f"dp{world} (one batch per GPU; dW summed over the ranks per vocabulary "
+                        f"slice with NCCL, overlapped with the next slice's GEMMs, {DP_COMM_SMS} SMs "
+                        f"left to the exchange)" if exchange else
+                        f"dp{world} (one batch per GPU, no collective on the data path)"),
         "l2": "inputs larger than L2 (W alone is %.2f GB)" % (V * wl.d * 2 / 1e9),
     }
 
@@ -335,8 +341,11 @@ class Problem:
     """One workload's device tensors and its forward + backward step through
     the public binding."""
 
-    def __init__(self, torch, sts, index, dev, rank, T=None, V=None):
+    def __init__(self, torch, sts, index, dev, rank, T=None, V=None, exchange=False):
         self.wl = wl = workloads.WORKLOADS[index]
+        # data-parallel training: every rank's dW is a partial sum, added over
+        # the ranks slice by slice as the backward writes it
+        self.red = sts.SliceAllReduce() if exchange and wl.backward else None
         self.data = data = workloads.make(index, batch=rank, T=T, V=V)
         self.T, self.d, self.V = data["H"].shape[0], wl.d, data["W"].shape[0]
         self.sts = sts
@@ -372,7 +381,10 @@ class Problem:
         lp, saved, _ = sts.sts_forward(Hx, self.W, yx, taux, kx, px, mux, ws=self.ws_f)
         if self.wl.backward:
             sts.sts_backward(Hx, self.W, yx, taux, kx, px, mux, saved, gx, dW=self.dW, dH=self.dH,
-                             vocab_chunk=self.wl.vocab_chunk, ws=self.ws_b)
+                             vocab_chunk=self.wl.vocab_chunk, ws=self.ws_b, on_dw_slice=self.red,
+                             comm_sms=DP_COMM_SMS if self.red is not None else 0)
+            if self.red is not None:
+                self.red.finish()
         return lp
 
     def check_status(self):
@@ -428,7 +440,9 @@ def run_ours(args, rank, local_rank, world):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     peaks = _peaks()
-    prob = Problem(torch, sts, args.workload, dev, rank, T=args.rows, V=args.vocab)
+    exchange = world > 1 and not args.no_dp_exchange
+    prob = Problem(torch, sts, args.workload, dev, rank, T=args.rows, V=args.vocab,
+                   exchange=exchange)
     wl, T, d, V, data = prob.wl, prob.T, prob.d, prob.V, prob.data
 
     for _ in range(args.warmup):
@@ -510,7 +524,7 @@ def run_ours(args, rank, local_rank, world):
     if args.workload != SECOND_WORKLOAD and not (args.rows or args.vocab) and not args.no_second:
         del prob, dbufs, host
         torch.cuda.empty_cache()
-        p2 = Problem(torch, sts, SECOND_WORKLOAD, dev, rank)
+        p2 = Problem(torch, sts, SECOND_WORKLOAD, dev, rank, exchange=exchange)
         for _ in range(args.warmup):
             p2.step()
         torch.cuda.synchronize()
@@ -523,7 +537,7 @@ def run_ours(args, rank, local_rank, world):
         launches_all += int(reduce_sum(launches2, dev))
         r2, r2_res = kernel_rooflines(kern2, args.steps, p2.T, p2.d, p2.V, peaks)
         second = {
-            "config": workload_config(p2.wl, p2.T, p2.V, world),
+            "config": workload_config(p2.wl, p2.T, p2.V, world, exchange=exchange),
             "value": round(world * p2.T / (ms2 / 1e3), 1), "unit": UNIT,
             "ms_per_step": round(ms2, 3), "steps": args.steps,
             "step_roofline": step_roofline(p2.wl, p2.T, p2.d, p2.V, ms2, peaks, clk2),
@@ -549,7 +563,8 @@ def run_ours(args, rank, local_rank, world):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
-            "config": workload_config(wl, T, V, world, reduced=bool(args.rows or args.vocab)),
+            "config": workload_config(wl, T, V, world, reduced=bool(args.rows or args.vocab),
+                                      exchange=exchange),
             "step_roofline": step_roofline(wl, T, d, V, ms_max, peaks, clk),
             "roofline": roof,
             "roofline_resolver": roof_res,
@@ -624,6 +639,8 @@ def main(argv=None):
                     help="skip the second timed workload (T=8192, d=4096, V=151936)")
     ap.add_argument("--rows", type=int, default=None,
                     help="override T (small profiling captures only; not a bench line)")
+    ap.add_argument("--no-dp-exchange", action="store_true",
+                    help="with --gpus N > 1, leave each rank's dW local (independent replicas)")
     ap.add_argument("--vocab", type=int, default=None,
                     help="override V (small profiling captures only; not a bench line)")
     args = ap.parse_args(argv)

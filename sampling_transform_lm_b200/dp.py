@@ -49,7 +49,8 @@ class SliceAllReduce:
             self.works.append((dist.all_reduce(dW_slice, group=self.group, async_op=True), dW_slice))
 
     def finish(self):
-        """Wait for every slice's exchange (on the device for CUDA tensors)."""
+        """Wait for every slice's exchange (on the device for CUDA tensors);
+        returns the slices (v0, rows) exchanged since the last call."""
         world = dist.get_world_size(self.group)
         for work, sl in self.works:
             work.wait()
@@ -58,4 +59,5 @@ class SliceAllReduce:
         if self.comm_stream is not None:
             torch.cuda.current_stream(self.comm_stream.device).wait_stream(self.comm_stream)
         self.works = []
-        return self.slices
+        done, self.slices = self.slices, []
+        return done
