@@ -77,6 +77,7 @@
 // degree-6 Taylor polynomial, whose truncation error (< 4e-19) is below half
 // an ulp. Elements in the clamped far-tail bucket use the library exp.
 #include <cfloat>
+#include <climits>
 #include <type_traits>
 #include <cmath>
 
@@ -136,6 +137,7 @@ struct RSmem {
   double bd[4];
   long long bl[4];
   int bi[4];
+  int row_next;       // the row this CTA resolves after the current one
   int ncand;
   int tcount[RT];     // gathered keys of each thread (slot j of thread t: cand[j RT + t])
 };
@@ -2226,12 +2228,33 @@ __global__ void __launch_bounds__(RT, 1) resolve_kernel(const ResolveArgs a) {
     h.p = a.top_p[row];
     h.mu = a.min_p[row];
   };
+  // Rows are handed out dynamically (their costs differ several-fold by
+  // metadata, and a static split leaves the launch waiting on its slowest
+  // CTA): the first gridDim.x rows go one per CTA, the rest in the order CTAs
+  // claim them from the header's counter. A CTA claims the row after next at
+  // the start of each row, so the atomic's latency overlaps the row's work and
+  // the next row's metadata can be loaded one row ahead.
+  unsigned long long claim = 0;
+  if (threadIdx.x == 0) sm.row_next = (int)gridDim.x + (int)atomicAdd(&a.hdr->next_row, 1ull);
+  __syncthreads();
+  int nxt = sm.row_next;
+  auto advance = [&]() {
+    if (threadIdx.x == 0) sm.row_next = (int)claim;
+    __syncthreads();
+    const int r2 = nxt;
+    nxt = sm.row_next;
+    return r2;
+  };
   Ahead ahead;
   load_ahead(blockIdx.x, ahead);
 
-  for (int r = blockIdx.x; r < a.rows; r += gridDim.x) {
+  for (int r = blockIdx.x; r < a.rows; r = advance()) {
     const Ahead cur = ahead;
-    load_ahead(r + gridDim.x, ahead);
+    if (threadIdx.x == 0) {
+      const unsigned long long c = atomicAdd(&a.hdr->next_row, 1ull) + gridDim.x;
+      claim = c < (unsigned long long)INT_MAX ? c : (unsigned long long)INT_MAX;
+    }
+    load_ahead(nxt, ahead);
     const float* __restrict__ x = a.S + (size_t)r * (size_t)a.ld;
     const bool invalid = (cur.flags & STS_ROW_INVALID) != 0;
     if (invalid) {
@@ -2435,6 +2458,8 @@ cudaError_t launch_resolve(const ResolveArgs& a, int num_sms, cudaStream_t strea
   if (e != cudaSuccess) return e;
   const int grid = a.rows < num_sms ? a.rows : num_sms;
   if (grid <= 0) return cudaSuccess;
+  e = cudaMemsetAsync(&a.hdr->next_row, 0, sizeof(a.hdr->next_row), stream);  // the row counter
+  if (e != cudaSuccess) return e;
   kern<<<grid, RT, smem, stream>>>(a);
   return cudaGetLastError();
 }

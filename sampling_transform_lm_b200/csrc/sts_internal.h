@@ -14,13 +14,16 @@ namespace sts {
 //   bad_row_code: min over failing rows of (row << 32 | status); all-ones = none
 //   err:          first non-row error (timeout, overflow), 0 = none
 //   path_rows:    rows the resolver decided by each path (diagnostic counters)
+//   next_row:     the resolver's row counter (rows handed out dynamically;
+//                 zeroed before every resolver launch)
 enum ResolvePath : int { kPathPlanned = 0, kPathFast = 1, kPathExact = 2, kPathIdentity = 3 };
 struct WsHeader {
   unsigned long long bad_row_code;
   int err;
   int pad0;
   unsigned long long path_rows[4];
-  unsigned long long reserved[26];
+  unsigned long long next_row;
+  unsigned long long reserved[25];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
