@@ -28,6 +28,10 @@
 //                 ~2e-6, well below the bf16 rounding of dz)
 //   kEpiStoreF32  acc -> fp32
 //   kEpiReduceF32 acc -> fp32, added in place (TMA reduce-add)
+//   kEpiStoreF32T, kEpiReduceF32T  the same into C's transpose: element
+//                 (m, n) lands at row n, column m of the output, so a
+//                 product computed as (dW)^T = H^T . dZ is written as dW
+//                 (its 32 x 32 blocks are staged transposed in shared memory)
 #pragma once
 
 #include "sts_device.cuh"
@@ -49,7 +53,14 @@ constexpr size_t GEMM_SMEM_BYTES =
     1024 + GEMM_STAGES * GEMM_STAGE_BYTES + GEMM_EPI_BYTES + 256;
 constexpr int GEMM_GROUP_M = 16;  // m-blocks per raster group (L2 reuse of B)
 
-enum EpiKind : int { kEpiLogits = 0, kEpiDZ = 1, kEpiStoreF32 = 2, kEpiReduceF32 = 3 };
+enum EpiKind : int {
+  kEpiLogits = 0,
+  kEpiDZ = 1,
+  kEpiStoreF32 = 2,
+  kEpiReduceF32 = 3,
+  kEpiStoreF32T = 4,
+  kEpiReduceF32T = 5
+};
 
 struct GemmParams {
   int M, N, K;
@@ -343,9 +354,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const uint32_t sb = smem_u32(stg + sel * GEMM_EPI_BUF);
         if (lane == 0) bulk_wait_read<1>();
         __syncwarp();
+        constexpr bool kT = (EPI == kEpiStoreF32T || EPI == kEpiReduceF32T);
         const uint32_t row_addr = sb + (uint32_t)lane * 128u;
+        if (kT) {
+          // block row j holds column ncol0 + j of the tile: lane's element goes
+          // to column `lane` of that row (128-byte swizzle: 16-byte chunk
+          // lane / 4 of row j sits at chunk (lane / 4) ^ (j % 8))
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+          for (int j = 0; j < 32; ++j)
+            st_shared_f32(sb + (uint32_t)j * 128u + ((uint32_t)((lane >> 2) ^ (j & 7)) << 4) +
+                              ((uint32_t)(lane & 3) << 2),
+                          v[j]);
+        }
+#pragma unroll
+        for (int c = 0; c < 8 && !kT; ++c) {
           uint32_t w0, w1, w2, w3;
           if (EPI == kEpiDZ) {
             w0 = pack_bf16x2(v[c * 8 + 0], v[c * 8 + 1]);
@@ -365,6 +387,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (lane == 0 && quarter_live) {
           if (EPI == kEpiReduceF32)
             tma_reduce_add_2d(&map_c, sb, p.c_x0 + ncol0, p.c_y0 + row0);
+          else if (EPI == kEpiReduceF32T)
+            tma_reduce_add_2d(&map_c, sb, p.c_x0 + row0, p.c_y0 + ncol0);
+          else if (EPI == kEpiStoreF32T)
+            tma_store_2d(&map_c, sb, p.c_x0 + row0, p.c_y0 + ncol0);
           else
             tma_store_2d(&map_c, sb, p.c_x0 + ncol0, p.c_y0 + row0);
           bulk_commit();

@@ -217,14 +217,33 @@ FwdLayout fwd_layout(const sts_shape* s) {
 }
 
 struct BwdLayout {
-  size_t dz_off, total;
+  size_t dz_off, ht_off, total;
+  int64_t ht_ld;  // row stride of H^T (elements): T rounded up to 8 (16-byte TMA rows)
 };
 
 BwdLayout bwd_layout(const sts_shape* s) {
   BwdLayout L;
   L.dz_off = kAlign;
-  L.total = align_up(L.dz_off + (size_t)s->T * (size_t)vocab_chunk(s) * 2, kAlign);
+  L.ht_ld = (s->T + 7) / 8 * 8;
+  L.ht_off = align_up(L.dz_off + (size_t)s->T * (size_t)vocab_chunk(s) * 2, kAlign);
+  L.total = align_up(L.ht_off + (size_t)s->d * (size_t)L.ht_ld * 2, kAlign);
   return L;
+}
+
+// HT[j][t] = H[t][j] (bf16), 32 x 32 tiles through shared memory.
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ H, int64_t T, int64_t d,
+                                      uint16_t* __restrict__ HT, int64_t ld) {
+  __shared__ uint16_t tile[32][33];
+  const int64_t t0 = (int64_t)blockIdx.y * 32, j0 = (int64_t)blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t t = t0 + i, j = j0 + threadIdx.x;
+    if (t < T && j < d) tile[i][threadIdx.x] = H[t * d + j];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t j = j0 + i, t = t0 + threadIdx.x;
+    if (j < d && t < T) HT[j * ld + t] = tile[threadIdx.x][i];
+  }
 }
 
 size_t filter_bytes(const sts_shape* s) { return align_up(sizeof(WsHeader) + (size_t)s->T * 4, kAlign); }
@@ -384,11 +403,21 @@ sts_status backward_impl(const sts_shape* shape, const void* H, const void* W,
   void* dZ = wsb + L.dz_off;
   STS_TRY(reset_header(ws, st));
 
-  CUtensorMap m_h_k, m_w_k, m_h_mn, m_w_mn, m_dw, m_dh;
+  // dW is formed as (dW)^T = H^T . dZ, so that its 128-row operand is
+  // K-major (H^T, transposed once per call) and only the 256-wide one (dZ)
+  // is read MN-major; the epilogue writes the product transposed, i.e. dW
+  void* HT = wsb + L.ht_off;
+  CUtensorMap m_h_k, m_w_k, m_ht_k, m_w_mn, m_dw, m_dh;
   if (!map_kmajor(&m_h_k, H, d, T, d, GEMM_BM) || !map_kmajor(&m_w_k, W, d, V, d, GEMM_BN) ||
-      !map_mnmajor(&m_h_mn, H, d, T, d) || !map_mnmajor(&m_w_mn, W, d, V, d) ||
+      !map_kmajor(&m_ht_k, HT, T, d, L.ht_ld, GEMM_BM) || !map_mnmajor(&m_w_mn, W, d, V, d) ||
       !map_out_f32(&m_dw, dW, d, V, d) || !map_out_f32(&m_dh, dH, d, T, d))
     return STS_ERR_CUDA;
+  STS_CUDA(timed_launch(STS_KERNEL_DW_GEMM, st, [&] {
+    const dim3 grid((unsigned)((d + 31) / 32), (unsigned)((T + 31) / 32));
+    transpose_bf16_kernel<<<grid, dim3(32, 8), 0, st>>>(static_cast<const uint16_t*>(H), T, d,
+                                                        static_cast<uint16_t*>(HT), L.ht_ld);
+    return cudaGetLastError();
+  }));
 
   for (int64_t v0 = 0; v0 < V; v0 += Vc) {
     const int64_t w = (V - v0) < Vc ? (V - v0) : Vc;
@@ -416,16 +445,18 @@ sts_status backward_impl(const sts_shape* shape, const void* H, const void* W,
       return run_gemm<false, false, kEpiDZ>(m_h_k, m_w_k, m_dz_out, p, dev.sms, st);
     }));
 
-    // 2. dW[v0:v0+w] = dZ^T . H (both operands MN-major), written once
+    // 2. dW[v0:v0+w] = (H^T . dZ)^T: H^T K-major, dZ MN-major, the tile
+    //    stored transposed; written once
     GemmParams q{};
-    q.M = (int)w;
-    q.N = (int)d;
+    q.M = (int)d;
+    q.N = (int)w;
     q.K = (int)T;
     q.c_y0 = (int)v0;
     q.err = &hdr->err;
     STS_CUDA(timed_launch(STS_KERNEL_DW_GEMM, st, [&] {
-      return accumulate_dW ? run_gemm<true, true, kEpiReduceF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st)
-                           : run_gemm<true, true, kEpiStoreF32>(m_dz_mn, m_h_mn, m_dw, q, dev.sms, st);
+      return accumulate_dW
+                 ? run_gemm<false, true, kEpiReduceF32T>(m_ht_k, m_dz_mn, m_dw, q, dev.sms, st)
+                 : run_gemm<false, true, kEpiStoreF32T>(m_ht_k, m_dz_mn, m_dw, q, dev.sms, st);
     }));
     // the slice is final once this GEMM completes on `st`: hand it out before
     // enqueuing the work that follows, so its exchange overlaps that work

@@ -51,8 +51,10 @@ def test_workspace_sizes(lib):
     flt = lib.sts_workspace_bytes(ctypes.byref(sh), 2)
     # forward: header + flags + one row chunk of fp32 logits (row stride padded to 4)
     assert fwd >= 1024 * 50000 * 4 and fwd % 1024 == 0
-    # backward: one vocab chunk (default 16384 columns) of bf16 dZ for all rows
-    assert lib.sts_vocab_chunk(ctypes.byref(sh)) == 16384 and bwd >= 1000 * 16384 * 2
+    # backward: one vocab chunk (default 16384 columns) of bf16 dZ for all rows,
+    # and H^T in bf16 (rows padded to 8 elements)
+    assert lib.sts_vocab_chunk(ctypes.byref(sh)) == 16384
+    assert bwd >= 1000 * 16384 * 2 + 128 * 1000 * 2
     assert flt >= 1000 * 4
     sh2 = _shape(T=1000, d=128, V=50000, vc=8192, rc=256)
     assert lib.sts_workspace_bytes(ctypes.byref(sh2), 1) < bwd
