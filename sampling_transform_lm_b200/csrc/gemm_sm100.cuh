@@ -86,6 +86,10 @@ struct GemmParams {
   int group_m;
 };
 
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ void gemm_tile_coords(int t, int num_m, int num_n, int group_m, int& mb,
                                                  int& nb) {
   const int per_group = group_m * num_n;
