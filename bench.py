@@ -637,7 +637,8 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": workload_config(wl, wl.T, wl.V, world),
+        "config": workload_config(wl, wl.T, wl.V, world,
+                                  exchange=world > 1 and not args.no_dp_exchange),
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
