@@ -1026,7 +1026,9 @@ __device__ __forceinline__ void append_hits(unsigned gm, unsigned long long* tbu
 // independent chains and summed into split accumulators, so float64 latency
 // is covered. Every lane of a warp runs every batch (invalid slots masked), so
 // the warp votes always see the full warp.
-template <bool VEC, bool NEED_Z, bool COUNTS>
+// TWO: the second gather range may be non-empty (false: compiled out, for the
+// top-p rows without min-p, the common case).
+template <bool VEC, bool NEED_Z, bool COUNTS, bool TWO = true>
 __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, int V, float m,
                                         const Plan2 pl, Pass2& P) {
   constexpr int E = 8;
@@ -1129,7 +1131,7 @@ __device__ __noinline__ void pass2_impl(RSmem& sm, const float* __restrict__ x, 
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const unsigned b = (unsigned)bb[e];
-      const bool g = ok(e) & ((b - g1s <= g1n) | (b - g2s <= g2n));
+      const bool g = TWO ? ok(e) & ((b - g1s <= g1n) | (b - g2s <= g2n)) : ok(e) & (b - g1s <= g1n);
       gm |= g ? 1u << e : 0u;
     }
     // each thread appends its hits to its own slots (no coordination between
@@ -1250,10 +1252,14 @@ __device__ void pass2(RSmem& sm, const float* __restrict__ x, int V, float m, bo
     else
       pass2_impl<VEC, false, true>(sm, x, V, m, pl, P);
   } else {
-    if (need_z)
-      pass2_impl<VEC, true, false>(sm, x, V, m, pl, P);
-    else
+    if (need_z) {
+      if (pl.g2_lo > pl.g2_hi && pl.b_mu < 0)
+        pass2_impl<VEC, true, false, false>(sm, x, V, m, pl, P);
+      else
+        pass2_impl<VEC, true, false>(sm, x, V, m, pl, P);
+    } else {
       pass2_impl<VEC, false, false>(sm, x, V, m, pl, P);
+    }
   }
 }
 
