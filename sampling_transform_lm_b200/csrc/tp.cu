@@ -236,7 +236,29 @@ __device__ __forceinline__ double unit_lo(int b) {
 }
 __device__ __forceinline__ double unit_hi(int b) { return exp(-(double)b / 128.0) * (1.0 + 1e-6); }
 
+// exp(s - m) in float64 for an element of bucket b (b = bin0(s, m)): the
+// bucket's factor exp(-b/128) from a per-CTA table times exp(r), r = (s - m)
+// + b/128 in [-1/128, 0], from its Taylor polynomial to degree 6 (truncation
+// below 4e-19, under half an ulp); the clamped last bucket takes the library
+// exp.
+constexpr size_t TP_EXACT_SMEM = NB * sizeof(double);
+
+__device__ __forceinline__ double tp_mass(const double* tab, float s, double md, int b) {
+  const double x = (double)s - md;
+  if (b >= NB - 1) return exp(x);
+  const double r = fma((double)b, 1.0 / 128.0, x);
+  double q = 1.0 / 720.0;
+  q = fma(q, r, 1.0 / 120.0);
+  q = fma(q, r, 1.0 / 24.0);
+  q = fma(q, r, 1.0 / 6.0);
+  q = fma(q, r, 0.5);
+  q = fma(q, r, 1.0);
+  q = fma(q, r, 1.0);
+  return tab[b] * q;
+}
+
 __global__ void __launch_bounds__(TP_RT) tp_exact_kernel(const TpExactArgs a) {
+  extern __shared__ __align__(16) double tp_tab[];  // exp(-b / 128), b < NB
   __shared__ TpRed red;
   __shared__ long long redl[TP_NW];
   __shared__ double redd[TP_NW];
@@ -244,6 +266,8 @@ __global__ void __launch_bounds__(TP_RT) tp_exact_kernel(const TpExactArgs a) {
   __shared__ int ngath;
   __shared__ int cnt_s[NB];
   const int tid = threadIdx.x;
+  for (int b = tid; b < NB; b += TP_RT) tp_tab[b] = exp(-(double)b / 128.0);
+  __syncthreads();
   for (int r = blockIdx.x; r < a.T; r += gridDim.x) {
     const float mr = a.m[r];
     const double md = (double)mr;
@@ -420,7 +444,7 @@ __global__ void __launch_bounds__(TP_RT) tp_exact_kernel(const TpExactArgs a) {
     for (int j = tid; j < a.Vl; j += TP_RT) {
       const float s = x[j];
       const int b = bin0(s, mr);
-      const double q = exp((double)s - md);
+      const double q = tp_mass(tp_tab, s, md, b);
       const unsigned long long K = ckey(s, (int)(a.off + j));
       z += q;
       if (b < bk) mbk += q;
@@ -479,12 +503,16 @@ struct TpFinishArgs {
   int32_t* need_gather;            // [T]: 1 where the bracket overflowed the sort
 };
 
-constexpr size_t TP_FINISH_SMEM = TP_SORT * (sizeof(unsigned long long) + sizeof(double));
+constexpr size_t TP_FINISH_SMEM =
+    TP_SORT * (sizeof(unsigned long long) + sizeof(double)) + NB * sizeof(double);
 
 __global__ void __launch_bounds__(TP_RT) tp_finish_kernel(const TpFinishArgs a) {
   extern __shared__ __align__(16) uint8_t tp_smem[];
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(tp_smem);
   double* scan = reinterpret_cast<double*>(tp_smem + TP_SORT * sizeof(unsigned long long));
+  double* tab = scan + TP_SORT;  // exp(-b / 128): the masses of the exact pass's stage
+  for (int b = threadIdx.x; b < NB; b += TP_RT) tab[b] = exp(-(double)b / 128.0);
+  __syncthreads();
   __shared__ TpRed red;
   __shared__ double redd[TP_NW];
   __shared__ int ntot_s;
@@ -558,11 +586,15 @@ __global__ void __launch_bounds__(TP_RT) tp_finish_kernel(const TpFinishArgs a) 
     {
       double run = 0.0;
       const int i0 = tid * per;
-      for (int i = i0; i < i0 + per && i < ntot; ++i) run += exp((double)ckey_value(keys[i]) - md);
+      auto qm = [&](int i) {
+        const float v = ckey_value(keys[i]);
+        return tp_mass(tab, v, md, bin0(v, mr));
+      };
+      for (int i = i0; i < i0 + per && i < ntot; ++i) run += qm(i);
       double total;
       double acc = tp_exscan<double>(run, redd, total);
       for (int i = i0; i < i0 + per && i < ntot; ++i) {
-        acc += exp((double)ckey_value(keys[i]) - md);
+        acc += qm(i);
         scan[i] = acc;
       }
     }
@@ -777,7 +809,10 @@ extern "C" sts_status sts_tp_exact(const float* S, int64_t T, int64_t Vl, int64_
   a.cand = reinterpret_cast<unsigned long long*>(cand);
   a.ncand = ncand;
   a.cap = (int)cap;
-  tp_exact_kernel<<<tp_grid(T), TP_RT, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  if (cudaFuncSetAttribute(tp_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)TP_EXACT_SMEM) != cudaSuccess)
+    return STS_ERR_CUDA;
+  tp_exact_kernel<<<tp_grid(T), TP_RT, TP_EXACT_SMEM, reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return cudaGetLastError() == cudaSuccess ? STS_OK : STS_ERR_CUDA;
 }
 
