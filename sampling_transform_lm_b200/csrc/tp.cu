@@ -70,6 +70,7 @@ __global__ void gather_shards_kernel(const float* __restrict__ src, int64_t worl
 constexpr int TP_RT = 512;            // threads per row CTA
 constexpr int TP_NW = TP_RT / 32;
 constexpr int TP_SORT = 8192;         // merged keys of a row sorted at once
+constexpr int TP_WINDOW = 2048;       // keys gathered around an estimated top-p crossing
 constexpr int TP_BPT = NB / TP_RT;    // buckets per thread in the plan scans
 
 // Per-row plan (int32 fields) and per-row float64 sums / keys of stage 3.
@@ -83,6 +84,7 @@ enum : int {
   kPlanRules = 6,   // bit 0 top-k, bit 1 top-p, bit 2 min-p
   kPlanFields = 8
 };
+// kSumZ is the total mass when top-k is off (unused, and partial, otherwise)
 enum : int { kSumZ = 0, kSumBk = 1, kSumLo = 2, kSumKept = 3, kSumKeptCnt = 4, kSumFields = 5 };
 enum : int { kKeyKept = 0, kKeyAll = 1, kKeyFields = 2 };
 
@@ -380,19 +382,21 @@ __global__ void __launch_bounds__(TP_RT) tp_exact_kernel(const TpExactArgs a) {
         for (int b = rlo; b <= rhi; ++b) n += cnt_s[b];
         int lo = rlo, hi = rhi;
         if (n > budget && rlo <= rhi) {
-          // the certain bracket does not fit: the widest run of buckets around
-          // the estimated crossing that does (the finish checks that it holds
-          // the crossing, else the row takes the gather form)
+          // the certain bracket does not fit: a run of buckets around the
+          // estimated crossing, grown to TP_WINDOW keys (the mid-bucket
+          // estimate is off by a bucket or two on flat rows; the finish checks
+          // that the run holds the crossing, else the row takes the gather form)
+          const long long want = budget < TP_WINDOW ? budget : TP_WINDOW;
           int c0 = (int)min(max((long long)hit[0], (long long)rlo), (long long)rhi);
           lo = hi = c0;
           n = cnt_s[c0];
           for (bool grew = true; grew;) {
             grew = false;
-            if (hi < rhi && n + cnt_s[hi + 1] <= budget) {
+            if (hi < rhi && n + cnt_s[hi + 1] <= want) {
               n += cnt_s[++hi];
               grew = true;
             }
-            if (lo > rlo && n + cnt_s[lo - 1] <= budget) {
+            if (lo > rlo && n + cnt_s[lo - 1] <= want) {
               n += cnt_s[--lo];
               grew = true;
             }
@@ -441,16 +445,23 @@ __global__ void __launch_bounds__(TP_RT) tp_exact_kernel(const TpExactArgs a) {
     double z = 0.0, mbk = 0.0, mlo = 0.0, mk = 0.0, ckept = 0.0;
     unsigned long long kkept = ~0ull, kall = ~0ull;
     unsigned long long* cand = a.cand + (size_t)r * (size_t)a.cap;
+    // the total mass is only used when top-k is off (the top-p target and
+    // identity rows); otherwise only the logits before the top-k bucket, the
+    // bracket and the min-p-kept ones are weighed
+    const bool zneed = !k_on;
     for (int j = tid; j < a.Vl; j += TP_RT) {
       const float s = x[j];
       const int b = bin0(s, mr);
-      const double q = tp_mass(tp_tab, s, md, b);
       const unsigned long long K = ckey(s, (int)(a.off + j));
-      z += q;
-      if (b < bk) mbk += q;
-      if (b < blo) mlo += q;
-      if (mu_on & (key32(s) >= kt)) {
-        mk += q;
+      const bool kept = mu_on & (key32(s) >= kt);
+      if (zneed | (b < bk) | (b < blo) | kept) {
+        const double q = tp_mass(tp_tab, s, md, b);
+        z += q;
+        if (b < bk) mbk += q;
+        if (b < blo) mlo += q;
+        if (kept) mk += q;
+      }
+      if (kept) {
         ckept += 1.0;
         kkept = K < kkept ? K : kkept;
       }
