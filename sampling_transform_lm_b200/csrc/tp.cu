@@ -28,8 +28,8 @@
 //      bracket (global token ids); sums are combined by sum, keys by min, the
 //      gathered keys by an all-gather;
 //      When the certain bracket holds more keys than one sort (flat rows),
-//      the widest run of its buckets around the crossing estimated from
-//      mid-bucket masses that fits is gathered instead;
+//      a run of its buckets around the crossing estimated from mid-bucket
+//      masses, up to TP_WINDOW keys, is gathered instead;
 //   4. every rank sorts the merged keys of each row, scans their float64
 //      masses from the mass before the gathered buckets and places the cuts
 //      exactly; a row whose crossing turns out to lie outside the gathered

@@ -18,9 +18,9 @@ Two forms of the forward, per row chunk:
   all-gather); every rank sorts and scans the merged keys and places the cuts.
   About 16 KB of counts plus the planned buckets' keys move per row, against
   4 V bytes of logits for the gather. Where the certain bracket holds more
-  keys than one sort, the buckets around the estimated crossing are gathered
-  and the finish checks that they hold it; rows it flags are resolved by the
-  gather form.
+  keys than one sort, up to 2048 keys around the estimated crossing are
+  gathered and the finish checks that they hold it; rows it flags are
+  resolved by the gather form.
 * ``gather``: the ranks' blocks are all-gathered, interleaved in rank order
   into full rows and the support program runs on them on every rank (the
   pages' form, with its full re-sort on every rank).
