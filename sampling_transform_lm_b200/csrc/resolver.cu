@@ -2095,6 +2095,9 @@ __device__ __noinline__ bool resolve_row_planned(RSmem& sm, const float* __restr
   const bool k_on = k >= 1 && k < V, p_on = p < 1.0f, mu_on = mu > 0.0f;
   sampled = false;
   if (!k_on && !p_on && !mu_on) return false;  // identity rows: the fast path's single pass
+  // top-p alone: no plan uses the sample, and the fast path's count pass
+  // streams the whole row faster than the sample's strided chunks
+  if (!k_on && !mu_on) return false;
   const int ns = sample_hist<VEC>(sm, x, V, m);
   sampled = true;
   const double scale = (double)V / (double)ns;
