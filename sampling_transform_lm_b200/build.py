@@ -18,7 +18,11 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsts.so")
 SOURCES = ["sts_api.cu", "resolver.cu", "noalloc.cu", "policy.cu", "tp.cu"]
-HEADERS = ["sts_device.cuh", "gemm_sm100.cuh", "sts_internal.h"]
+
+
+def _headers() -> list:
+    # every header of the sources: a change to any of them rebuilds the library
+    return sorted(f for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
 
 
 def _nvcc() -> str:
@@ -32,7 +36,7 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
+    deps = [os.path.join(CSRC, f) for f in SOURCES + _headers()]
     deps.append(os.path.join(ROOT, "include", "sts.h"))
     return any(os.path.getmtime(p) > t for p in deps)
 

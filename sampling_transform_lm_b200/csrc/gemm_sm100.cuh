@@ -332,21 +332,45 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (j < valid) tile_max = fmaxf(tile_max, v[j]);
         } else if (EPI == kEpiDZ) {
           if (coef != 0.f) {
+            static_assert(CW % 32 == 0, "a chunk is whole 32-column halves");
             const long long col0 = (long long)p.col_base + ncol0;
+            const long long yrel = y - col0;
+            const int yj = (yrel >= 0 && yrel < CW) ? (int)yrel : -1;  // onehot column
+            // z * (1/tau) is within 2 ulp of the forward's IEEE quotient; only
+            // values that close to the cut ("near") are re-divided exactly, so
+            // the membership decision is the forward's bit for bit. They are
+            // rare and take a separate pass, so the main loop carries no
+            // per-element branch and the exponentials of 32 columns overlap.
 #pragma unroll
-            for (int j = 0; j < CW; ++j) {
-              // z * (1/tau) is within 2 ulp of the forward's IEEE quotient; only
-              // values that close to the cut are re-divided exactly, so the
-              // membership decision is the forward's bit for bit
-              float sf = v[j] * rtau;
-              const long long col = col0 + j;
-              bool member = sf > cut_hi;
-              if (!member && sf >= cut_lo) {
-                sf = __fdiv_rn(v[j], tau);
-                member = (sf > cut) || (sf == cut && col <= (long long)cut_id);
+            for (int h = 0; h < CW; h += 32) {
+              uint32_t near = 0u;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const float sf = v[h + j] * rtau;
+                near |= ((sf >= cut_lo) & !(sf > cut_hi) ? 1u : 0u) << j;
               }
-              const float pr = member ? __expf(sf - lse) : 0.f;
-              v[j] = coef * ((col == y ? 1.f : 0.f) - pr);
+              // the near columns one at a time (a rolled loop: one copy of the
+              // exact division, and no register pressure on the main loop)
+              for (uint32_t todo = near; todo != 0u; todo &= todo - 1u) {
+                const int j0 = __ffs(todo) - 1;
+                float z = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) z = j == j0 ? v[h + j] : z;
+                const float sf = __fdiv_rn(z, tau);
+                const bool member =
+                    (sf > cut) || (sf == cut && col0 + h + j0 <= (long long)cut_id);
+                const float pr = member ? __expf(sf - lse) : 0.f;
+                const float o = coef * ((h + j0 == yj ? 1.f : 0.f) - pr);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[h + j] = j == j0 ? o : v[h + j];
+              }
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const float sf = v[h + j] * rtau;
+                const float pr = sf > cut_hi ? __expf(sf - lse) : 0.f;
+                const float out = coef * ((h + j == yj ? 1.f : 0.f) - pr);
+                v[h + j] = ((near >> j) & 1u) ? v[h + j] : out;
+              }
             }
           } else {
 #pragma unroll
