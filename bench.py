@@ -261,10 +261,12 @@ SECOND_WORKLOAD = 3  # T=8192, d=4096, V=151936: the other reading of "config 3"
 
 
 def vocab_chunk_label(wl, V):
-    """The backward's vocabulary chunk for this workload (the library's rule:
-    the workload's chunk, else 16384, clamped to V rounded up to 256)."""
-    vc = wl.vocab_chunk or 16384
-    return min(vc, (V + 255) // 256 * 256)
+    """The backward's vocabulary chunk for this workload, as the library picks
+    it (the workload's chunk, else its default, clamped to V rounded up to
+    256); a host-only call."""
+    import sampling_transform_lm_b200 as sts
+
+    return sts.sts_vocab_chunk(wl.T, wl.d, V, vocab_chunk=wl.vocab_chunk)
 
 
 DP_COMM_SMS = 8  # SMs the persistent backward GEMMs leave to the dW exchange (N > 1)

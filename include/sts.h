@@ -83,7 +83,7 @@ typedef struct {
   int64_t T;           /* rows (scored tokens), >= 1 */
   int64_t d;           /* hidden size, >= 8, multiple of 8 */
   int64_t V;           /* vocabulary size, >= 1, < 2^31 */
-  int64_t vocab_chunk; /* backward vocab chunk (multiple of 256); 0: 16384 */
+  int64_t vocab_chunk; /* backward vocab chunk (multiple of 256); 0: 28416 */
   int64_t row_chunk;   /* forward row chunk (multiple of 128); 0: default */
 } sts_shape;
 
@@ -117,7 +117,7 @@ typedef struct {
 size_t sts_workspace_bytes(const sts_shape* shape, int pass);
 
 /* The vocabulary chunk the backward uses for this shape: shape->vocab_chunk,
- * or 16384 when it is 0, clamped to V rounded up to 256. A pure function of
+ * or 28416 when it is 0, clamped to V rounded up to 256. A pure function of
  * the shape (workspace sizes do not depend on the device). Returns -1 for an
  * invalid shape. Not from the pages: they chunk the vocabulary but fix no
  * chunk size. */

@@ -283,7 +283,7 @@ def sts_workspace_bytes(T, d, V, pass_, vocab_chunk=0, row_chunk=0) -> int:
 
 
 def sts_vocab_chunk(T, d, V, vocab_chunk=0) -> int:
-    """The backward's vocabulary chunk for this shape (16384 when
+    """The backward's vocabulary chunk for this shape (28416 when
     ``vocab_chunk`` is 0; clamped to V rounded up to 256)."""
     sh = _shape(T, d, V, vocab_chunk, 0)
     n = load().sts_vocab_chunk(ctypes.byref(sh))

@@ -24,7 +24,11 @@
 namespace sts {
 namespace {
 
-constexpr int64_t kDefaultVocabChunk = 16384;
+// 111 x 256 columns: for T and d multiples of 512 the dz GEMM (ceil(T/128) x
+// Vc/256 tiles) and the dW GEMM (ceil(d/128) x Vc/256 tiles) then fill whole
+// waves of a 148-SM part (111 = 3 x 37), and a chunk this wide needs few launches
+// (six at V = 152,064; the bf16 dZ buffer is T x Vc x 2 bytes, 0.93 GB at T = 16384).
+constexpr int64_t kDefaultVocabChunk = 28416;
 constexpr size_t kDefaultChunkBytes = size_t(4) << 30;  // forward logits chunk budget
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -51,10 +51,10 @@ def test_workspace_sizes(lib):
     flt = lib.sts_workspace_bytes(ctypes.byref(sh), 2)
     # forward: header + flags + one row chunk of fp32 logits (row stride padded to 4)
     assert fwd >= 1024 * 50000 * 4 and fwd % 1024 == 0
-    # backward: one vocab chunk (default 16384 columns) of bf16 dZ for all rows,
+    # backward: one vocab chunk (default 28416 columns) of bf16 dZ for all rows,
     # and H^T in bf16 (rows padded to 8 elements)
-    assert lib.sts_vocab_chunk(ctypes.byref(sh)) == 16384
-    assert bwd >= 1000 * 16384 * 2 + 128 * 1000 * 2
+    assert lib.sts_vocab_chunk(ctypes.byref(sh)) == 28416
+    assert bwd >= 1000 * 28416 * 2 + 128 * 1000 * 2
     assert flt >= 1000 * 4
     sh2 = _shape(T=1000, d=128, V=50000, vc=8192, rc=256)
     assert lib.sts_workspace_bytes(ctypes.byref(sh2), 1) < bwd
@@ -159,7 +159,7 @@ def test_vocab_chunk_choice():
     for T, d, V in [(16384, 5120, 152064), (8192, 4096, 151936), (32768, 4096, 262144),
                     (4096, 2048, 32768), (300, 64, 100000)]:
         vc = sts.sts_vocab_chunk(T, d, V)
-        assert vc == min(16384, (V + 255) // 256 * 256)
+        assert vc == min(28416, (V + 255) // 256 * 256)
         assert sts.sts_vocab_chunk(T, d, V, vocab_chunk=8192) == 8192  # an explicit chunk is kept
         assert sts.sts_workspace_bytes(T, d, V, 1) >= T * vc * 2  # the workspace follows it
     assert sts.sts_vocab_chunk(64, 128, 1000) == 1024
