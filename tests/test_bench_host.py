@@ -133,3 +133,19 @@ def test_recorded_traffic_per_row_scales_to_the_average_launch(tmp_path, monkeyp
     assert bench.recorded_traffic(8, 4, 16, "resolve") is None    # launches unknown
     (csrc / "resolver.cu").write_text("int changed = 2;\n")
     assert bench.recorded_traffic(8, 4, 16, "resolve", 2) is None
+
+
+def test_config_names_the_chunk_the_library_picks():
+    import sampling_transform_lm_b200 as sts
+    import workloads
+
+    wl4, wl3 = workloads.WORKLOADS[4], workloads.WORKLOADS[3]
+    cfg = bench.workload_config(wl4, wl4.T, wl4.V, 1)
+    # the library's default for the headline shape: 111 x 256 columns
+    assert cfg["vocab_chunk"] == sts.sts_vocab_chunk(wl4.T, wl4.d, wl4.V) == 28416
+    assert (wl4.T // 128) * (cfg["vocab_chunk"] // 256) % 148 == 0  # dz tiles: whole waves
+    assert (wl4.d // 128) * (cfg["vocab_chunk"] // 256) % 148 == 0  # dW tiles: whole waves
+    # a workload that states its chunk keeps it; a small vocabulary clamps it
+    assert bench.workload_config(wl3, wl3.T, wl3.V, 1)["vocab_chunk"] == 8192
+    wl1 = workloads.WORKLOADS[1]
+    assert bench.workload_config(wl1, wl1.T, wl1.V, 1)["vocab_chunk"] == 1024
