@@ -77,7 +77,9 @@ def recorded_traffic(T, d, V, kernel, launches_per_step=None):
     ncu capture of this workload (profiles/dram_traffic_T*_d*_V*.json), or
     None when there is none or the kernel's sources changed since. A record
     kept per row (the resolver's: its traffic grows with the rows a launch
-    resolves) is scaled to the average launch, T / launches_per_step rows."""
+    resolves) is scaled to the average launch, T / launches_per_step rows; one
+    kept per logit (the projection's) to T / launches_per_step rows of V
+    logits; a full-chunk backward launch to the average launch's FLOPs."""
     import hashlib
     path = os.path.join(ROOT, "profiles", f"dram_traffic_T{T}_d{d}_V{V}.json")
     if not os.path.exists(path):
@@ -96,7 +98,15 @@ def recorded_traffic(T, d, V, kernel, launches_per_step=None):
         if not launches_per_step:
             return None
         return int(k["dram_bytes_per_row"] * T / launches_per_step)
-    return int(k["dram_read_bytes_per_launch"] + k["dram_write_bytes_per_launch"])
+    if "dram_bytes_per_logit" in k:  # the projection: its launches cover row chunks of full rows
+        if not launches_per_step:
+            return None
+        return int(k["dram_bytes_per_logit"] * (T / launches_per_step) * V)
+    full = k["dram_read_bytes_per_launch"] + k["dram_write_bytes_per_launch"]
+    if launches_per_step and "capture_flops" in k:
+        # a full-chunk launch, scaled to the step's average launch by its FLOPs
+        return int(full * (2.0 * T * d * V / launches_per_step) / k["capture_flops"])
+    return int(full)
 
 
 def dist_env():
@@ -421,7 +431,7 @@ def kernel_rooflines(kern, steps, T, d, V, peaks):
         roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
                 "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
                 "frac": round(achieved / peaks["bf16_sustained"], 4),
-                "traffic": recorded_traffic(T, d, V, dom),
+                "traffic": recorded_traffic(T, d, V, dom, dom_n / steps),
                 "launches": dom_n, "ms_per_step": round(dom_ms / steps, 3),
                 "frac_of_datasheet_dense_bf16": round(achieved / DATASHEET_BF16_TFLOPS, 4),
                 "peak_note": f"bf16 sustained ({peaks['source']}); kernel timed inside a long step"}

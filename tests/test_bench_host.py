@@ -149,3 +149,28 @@ def test_config_names_the_chunk_the_library_picks():
     assert bench.workload_config(wl3, wl3.T, wl3.V, 1)["vocab_chunk"] == 8192
     wl1 = workloads.WORKLOADS[1]
     assert bench.workload_config(wl1, wl1.T, wl1.V, 1)["vocab_chunk"] == 1024
+
+
+def test_recorded_gemm_traffic_scales_to_the_average_launch(tmp_path, monkeypatch):
+    import hashlib
+    csrc = tmp_path / "sampling_transform_lm_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    h = hashlib.sha256()
+    for name in bench._TRAFFIC_SOURCES["gemm"]:
+        (csrc / name).write_text(f"int {name.split('.')[0]} = 1;\n")
+        h.update(bench.source_code_only((csrc / name).read_text()).encode())
+    (tmp_path / "profiles").mkdir()
+    T, d, V = 8, 4, 16
+    rec = {"sources": {"gemm": h.hexdigest()[:16]},
+           "kernels": {"logits_gemm": {"dram_bytes_per_logit": 10.0},
+                       "dw_gemm": {"dram_read_bytes_per_launch": 900,
+                                   "dram_write_bytes_per_launch": 100,
+                                   "capture_flops": 2 * T * d * 8}}}
+    (tmp_path / "profiles" / f"dram_traffic_T{T}_d{d}_V{V}.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    # projection: 8 rows over 2 launches, 16 logits each, 10 bytes per logit
+    assert bench.recorded_traffic(T, d, V, "logits_gemm", 2) == 4 * 16 * 10
+    assert bench.recorded_traffic(T, d, V, "logits_gemm") is None
+    # a full-chunk launch (8 columns) scaled to the average of 4 launches over V = 16
+    assert bench.recorded_traffic(T, d, V, "dw_gemm") == 1000
+    assert bench.recorded_traffic(T, d, V, "dw_gemm", 4) == 500
